@@ -1,0 +1,297 @@
+/*
+ * CPU oracle for the pack -> attend -> unpack pipeline of
+ * "Dispatch-Aware Ragged Attention for Pruned Vision Transformers".
+ *
+ * TEST INFRASTRUCTURE ONLY.  This file is the plain, slow, fp64 statement of
+ * what the pipeline computes.  Only the test suite, the smoke check and the
+ * benchmark's CPU-baseline leg may load it; the product path never does.  It
+ * shares no code, header, table or helper with the CUDA library: every step
+ * (survivor bookkeeping, byte copies, format decoding, attention) is written
+ * out here on its own.
+ *
+ * Sources, by page and section:
+ *  - survivor bookkeeping and the packed layout: radpulse article, section
+ *    "Integrated pack pipeline, 2.24x end-to-end" (cu_seqlens is computed
+ *    first, survivors are copied into one contiguous flat tensor, the CLS
+ *    token is extracted at the end), and its section on the FA2 dispatch
+ *    ceiling (survivors packed into a contiguous ragged buffer, varlen API);
+ *  - attention: abstract (bidirectional attention kernel over the ragged
+ *    sequences) and the radpulse section "Bypassing the binding" (no causal
+ *    mask, no KV cache): for each sequence b and head h,
+ *        O = softmax(scale * Q K^T) V   over the L_b rows of sequence b.
+ *    The softmax scale 1/sqrt(64) is the usual one; the pages do not print it.
+ *
+ * Conventions (readings of the pages where they are silent):
+ *  - index 0 (CLS) of every image is kept whatever the mask says;
+ *  - any nonzero mask byte means "keep";
+ *  - a packed sequence keeps ascending original token order, so CLS is the
+ *    first row of every packed sequence;
+ *  - scatter-unpack writes kept rows only and leaves dropped rows untouched.
+ *
+ * Build: gcc -O2 -shared -fPIC -pthread ragged_oracle.c -lm   (no fast-math).
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#include <unistd.h>
+
+enum { OR_F16 = 0, OR_BF16 = 1, OR_F32 = 2, OR_F64 = 3 };
+
+/* ------------------------------------------------------------------------ */
+/* Survivor bookkeeping: keep mask -> cu_seqlens and source rows.            */
+/* ------------------------------------------------------------------------ */
+
+static int is_kept(const uint8_t *keep, int64_t L_full, int64_t b, int64_t j)
+{
+    if (j == 0)
+        return 1; /* CLS is always kept */
+    return keep[b * L_full + j] != 0;
+}
+
+/* cu[0] = 0, cu[b+1] = cu[b] + (number of kept tokens of image b).
+ * src_idx (optional) receives, for every packed row t, the flat dense row
+ * b * L_full + j it comes from.  Returns T = cu[B]. */
+int64_t oracle_seqlens(const uint8_t *keep, int64_t B, int64_t L_full,
+                       int32_t *cu, int32_t *src_idx)
+{
+    int64_t t = 0;
+    cu[0] = 0;
+    for (int64_t b = 0; b < B; ++b) {
+        for (int64_t j = 0; j < L_full; ++j) {
+            if (is_kept(keep, L_full, b, j)) {
+                if (src_idx)
+                    src_idx[t] = (int32_t)(b * L_full + j);
+                ++t;
+            }
+        }
+        cu[b + 1] = (int32_t)t;
+    }
+    return t;
+}
+
+/* Pack: packed row t = dense row of the t-th survivor, bytes copied as is. */
+int64_t oracle_pack(const uint8_t *dense, int64_t B, int64_t L_full, int64_t row_bytes,
+                    const uint8_t *keep, uint8_t *packed, int32_t *cu)
+{
+    int64_t t = 0;
+    cu[0] = 0;
+    for (int64_t b = 0; b < B; ++b) {
+        for (int64_t j = 0; j < L_full; ++j) {
+            if (is_kept(keep, L_full, b, j)) {
+                memcpy(packed + t * row_bytes, dense + (b * L_full + j) * row_bytes,
+                       (size_t)row_bytes);
+                ++t;
+            }
+        }
+        cu[b + 1] = (int32_t)t;
+    }
+    return t;
+}
+
+/* CLS extraction: cls row b = packed row cu[b]. */
+void oracle_unpack_cls(const uint8_t *packed, const int32_t *cu, int64_t B,
+                       int64_t row_bytes, uint8_t *cls)
+{
+    for (int64_t b = 0; b < B; ++b)
+        memcpy(cls + b * row_bytes, packed + (int64_t)cu[b] * row_bytes, (size_t)row_bytes);
+}
+
+/* Scatter back: dense_out[b, j] = packed row of survivor (b, j); rows of
+ * dropped tokens are not written. */
+void oracle_unpack(const uint8_t *packed, const uint8_t *keep, int64_t B, int64_t L_full,
+                   int64_t row_bytes, uint8_t *dense_out)
+{
+    int64_t t = 0;
+    for (int64_t b = 0; b < B; ++b) {
+        for (int64_t j = 0; j < L_full; ++j) {
+            if (is_kept(keep, L_full, b, j)) {
+                memcpy(dense_out + (b * L_full + j) * row_bytes, packed + t * row_bytes,
+                       (size_t)row_bytes);
+                ++t;
+            }
+        }
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* Exact widening of the stored formats to double.                          */
+/* ------------------------------------------------------------------------ */
+
+/* IEEE 754 binary16: 1 sign bit, 5 exponent bits (bias 15), 10 fraction bits. */
+static double half_to_double(uint16_t h)
+{
+    int sign = h >> 15;
+    int e = (h >> 10) & 0x1f;
+    int f = h & 0x3ff;
+    double v;
+    if (e == 0)
+        v = ldexp((double)f, -24);                 /* zero or subnormal: f * 2^-24 */
+    else if (e == 31)
+        v = f ? NAN : INFINITY;
+    else
+        v = ldexp((double)(0x400 | f), e - 25);    /* (1024 + f) * 2^(e - 15 - 10) */
+    return sign ? -v : v;
+}
+
+/* bfloat16 is the upper half of an IEEE binary32. */
+static double bfloat_to_double(uint16_t h)
+{
+    uint32_t u = (uint32_t)h << 16;
+    float x;
+    memcpy(&x, &u, sizeof x);
+    return (double)x;
+}
+
+static double load_elem(const void *base, int dtype, int64_t idx)
+{
+    switch (dtype) {
+    case OR_F16: return half_to_double(((const uint16_t *)base)[idx]);
+    case OR_BF16: return bfloat_to_double(((const uint16_t *)base)[idx]);
+    case OR_F32: return (double)((const float *)base)[idx];
+    default: return ((const double *)base)[idx];
+    }
+}
+
+void oracle_decode(const void *src, int dtype, int64_t n, double *dst)
+{
+    for (int64_t i = 0; i < n; ++i)
+        dst[i] = load_elem(src, dtype, i);
+}
+
+/* ------------------------------------------------------------------------ */
+/* Attention over each packed sequence, in double.                          */
+/* ------------------------------------------------------------------------ */
+
+typedef struct {
+    const void *q, *k, *v;
+    int dtype;
+    int64_t tok_stride, head_stride;     /* elements */
+    const int32_t *cu;
+    const int32_t *seqs;                 /* sequences to compute */
+    int64_t n_seqs, H, d;
+    double scale;
+    double *out;                         /* [T, H, d] doubles */
+    int64_t next;                        /* shared work counter */
+    int failed;
+} attn_job;
+
+/* One (sequence, head): for every query row i,
+ *   s_j = scale * <q_i, k_j>,  m = max_j s_j,
+ *   p_j = exp(s_j - m) / sum_j' exp(s_j' - m),
+ *   o_i = sum_j p_j v_j. */
+static int attend_one(attn_job *J, int64_t b, int64_t h)
+{
+    const int64_t start = J->cu[b];
+    const int64_t L = (int64_t)J->cu[b + 1] - start;
+    const int64_t d = J->d;
+    if (L <= 0)
+        return 0;
+    double *Q = malloc(sizeof(double) * (size_t)(L * d));
+    double *K = malloc(sizeof(double) * (size_t)(L * d));
+    double *V = malloc(sizeof(double) * (size_t)(L * d));
+    double *s = malloc(sizeof(double) * (size_t)L);
+    if (!Q || !K || !V || !s) {
+        free(Q); free(K); free(V); free(s);
+        return -1;
+    }
+    for (int64_t i = 0; i < L; ++i) {
+        for (int64_t c = 0; c < d; ++c) {
+            int64_t idx = (start + i) * J->tok_stride + h * J->head_stride + c;
+            Q[i * d + c] = load_elem(J->q, J->dtype, idx);
+            K[i * d + c] = load_elem(J->k, J->dtype, idx);
+            V[i * d + c] = load_elem(J->v, J->dtype, idx);
+        }
+    }
+    for (int64_t i = 0; i < L; ++i) {
+        double m = -INFINITY;
+        for (int64_t j = 0; j < L; ++j) {
+            double dot = 0.0;
+            for (int64_t c = 0; c < d; ++c)
+                dot += Q[i * d + c] * K[j * d + c];
+            s[j] = J->scale * dot;
+            if (s[j] > m)
+                m = s[j];
+        }
+        double l = 0.0;
+        for (int64_t j = 0; j < L; ++j) {
+            s[j] = exp(s[j] - m);
+            l += s[j];
+        }
+        double *o = J->out + ((start + i) * J->H + h) * d;
+        for (int64_t c = 0; c < d; ++c) {
+            double acc = 0.0;
+            for (int64_t j = 0; j < L; ++j)
+                acc += s[j] * V[j * d + c];
+            o[c] = acc / l;
+        }
+    }
+    free(Q); free(K); free(V); free(s);
+    return 0;
+}
+
+static void *attn_worker(void *arg)
+{
+    attn_job *J = (attn_job *)arg;
+    for (;;) {
+        int64_t item = __atomic_fetch_add(&J->next, 1, __ATOMIC_RELAXED);
+        if (item >= J->n_seqs * J->H)
+            break;
+        int64_t b = J->seqs[item / J->H];
+        int64_t h = item % J->H;
+        if (attend_one(J, b, h) != 0)
+            __atomic_store_n(&J->failed, 1, __ATOMIC_RELAXED);
+    }
+    return NULL;
+}
+
+int oracle_num_cores(void)
+{
+    long n = sysconf(_SC_NPROCESSORS_ONLN);
+    return n > 0 ? (int)n : 1;
+}
+
+/* q, k, v: element pointers of the packed arrays (rows cu[b]..cu[b+1]-1 of
+ * sequence b), token stride and head stride in elements, all three sharing the
+ * same strides (separate arrays or views into one fused array).
+ * seqs/n_seqs: the sequences to compute (NULL: all B); out rows of other
+ * sequences are left untouched.  threads <= 0: one per online core.
+ * Returns 0, or -1 if a buffer could not be allocated. */
+int oracle_attention(const void *q, const void *k, const void *v, int dtype,
+                     int64_t tok_stride, int64_t head_stride, const int32_t *cu, int64_t B,
+                     int64_t H, int64_t d, double scale, const int32_t *seqs, int64_t n_seqs,
+                     double *out, int threads)
+{
+    int32_t *all = NULL;
+    if (!seqs) {
+        all = malloc(sizeof(int32_t) * (size_t)(B > 0 ? B : 1));
+        if (!all)
+            return -1;
+        for (int64_t b = 0; b < B; ++b)
+            all[b] = (int32_t)b;
+        seqs = all;
+        n_seqs = B;
+    }
+    attn_job J = {q, k, v, dtype, tok_stride, head_stride, cu, seqs, n_seqs, H, d,
+                  scale, out, 0, 0};
+    if (threads <= 0)
+        threads = oracle_num_cores();
+    if (threads == 1) {
+        attn_worker(&J);
+    } else {
+        pthread_t *tid = malloc(sizeof(pthread_t) * (size_t)threads);
+        int started = 0;
+        if (tid) {
+            for (; started < threads - 1; ++started)
+                if (pthread_create(&tid[started], NULL, attn_worker, &J) != 0)
+                    break;
+        }
+        attn_worker(&J); /* the calling thread works too; finishes any leftovers */
+        for (int i = 0; i < started; ++i)
+            pthread_join(tid[i], NULL);
+        free(tid);
+    }
+    free(all);
+    return J.failed ? -1 : 0;
+}

@@ -1,0 +1,83 @@
+"""Plant mistakes in a copy of the CPU oracle and check that the pins catch each one.
+
+Every mutant is a plausible slip in the oracle's C source (a dropped term, a
+wrong sign, a transposed operand, a lost index, a missed convention).  The
+mutant is compiled on the CPU into a temporary library, swapped in for the
+real oracle, and the pin tests of ``test_oracle_pins`` are run against it;
+at least one must fail.  No GPU is involved.
+"""
+import os
+import subprocess
+
+import numpy as np
+import pytest
+
+import oracle
+import test_oracle_pins as pins
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "ragged_oracle.c")
+
+MUTANTS = {
+    "cls_not_forced": ("if (j == 0)\n        return 1;", "if (j < 0)\n        return 1;"),
+    "scale_dropped": ("s[j] = J->scale * dot;", "s[j] = dot;"),
+    "qk_transposed": ("dot += Q[i * d + c] * K[j * d + c];", "dot += Q[j * d + c] * K[i * d + c];"),
+    "last_value_dropped": ("for (int64_t j = 0; j < L; ++j)\n                acc += s[j] * V[j * d + c];",
+                           "for (int64_t j = 0; j < L - 1; ++j)\n                acc += s[j] * V[j * d + c];"),
+    "not_normalised": ("o[c] = acc / l;", "o[c] = acc;"),
+    "exp_sign_flipped": ("s[j] = exp(s[j] - m);", "s[j] = exp(m - s[j]);"),
+    "head_offset_lost": ("(start + i) * J->tok_stride + h * J->head_stride + c;",
+                         "(start + i) * J->tok_stride + c;"),
+    "half_exponent_bias": ("ldexp((double)(0x400 | f), e - 25)", "ldexp((double)(0x400 | f), e - 24)"),
+    "cu_off_by_one": ("        cu[b + 1] = (int32_t)t;\n    }\n    return t;\n}\n\n/* Pack",
+                      "        cu[b + 1] = (int32_t)t + 1;\n    }\n    return t;\n}\n\n/* Pack"),
+    "pack_reads_wrong_row": ("dense + (b * L_full + j) * row_bytes,\n                       (size_t)row_bytes);\n                ++t;\n            }\n        }\n        cu[b + 1]",
+                             "dense + (b * L_full + (L_full - 1 - j)) * row_bytes,\n                       (size_t)row_bytes);\n                ++t;\n            }\n        }\n        cu[b + 1]"),
+}
+
+
+def _pin_calls():
+    calls = [pins.test_hand_example_seqlens_and_pack, pins.test_decode_f16_all_bit_patterns,
+             pins.test_decode_bf16_all_bit_patterns, pins.test_weights_sum_to_one,
+             pins.test_closed_forms, pins.test_hand_example_attention,
+             pins.test_brute_force_tiny_lengths, pins.test_attention_no_pruning_equals_dense_sdpa,
+             pins.test_key_shift_invariance_and_convex_hull]
+    for dt in ("f16", "bf16", "f32"):
+        calls.append(lambda dt=dt: pins.test_attention_equals_padded_masked_sdpa(dt))
+    for keep in pins._random_masks():
+        calls.append(lambda keep=keep: pins.test_seqlens_matches_flatnonzero(keep))
+        calls.append(lambda keep=keep: pins.test_pack_unpack_roundtrip(keep))
+    return calls
+
+
+@pytest.fixture(scope="module")
+def source():
+    return open(SRC).read()
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_mutant(name, source, tmp_path):
+    old, new = MUTANTS[name]
+    assert source.count(old) == 1, f"mutation site for {name} not found exactly once"
+    mutant_src = tmp_path / f"{name}.c"
+    mutant_src.write_text(source.replace(old, new))
+    so = tmp_path / f"lib{name}.so"
+    subprocess.run(["gcc", "-O2", "-std=c11", "-shared", "-fPIC", "-pthread", str(mutant_src),
+                    "-o", str(so), "-lm"], check=True)
+    real = oracle._load()
+    oracle.use_library(oracle.bind(str(so)))
+    caught = 0
+    try:
+        with np.errstate(all="ignore"):
+            for call in _pin_calls():
+                try:
+                    call()
+                except AssertionError:
+                    caught += 1
+    finally:
+        oracle.use_library(real)
+    assert caught > 0, f"no pin caught mutant {name}"
+
+
+def test_unmutated_source_passes_all_pins():
+    for call in _pin_calls():
+        call()
