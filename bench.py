@@ -1,0 +1,527 @@
+"""Benchmark of the ragged pack -> attend -> CLS pipeline on one or more B200s.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Workload: the serving regime of "Dispatch-Aware Ragged Attention for Pruned
+Vision Transformers" (abstract: BS=1-4; radpulse sections on the dispatch
+floor): DeiT-S shapes (197 tokens, 6 heads, head_dim 64, f16), batch sizes
+B in {1, 2, 4} and pruning rates {0, 25, 50, 80}% with +-10 points of
+per-image jitter.  One step is twelve calls, one per (B, rate); a call is the
+whole pipeline (pack with cu_seqlens, ragged attention with the CLS rows
+extracted in its epilogue) through the C ABI, followed by a stream
+synchronisation, so the time per call is host dispatch + device time.
+
+The reported value is microseconds per call (lower is better), over all
+calls of all ranks (with N GPUs each rank runs an independent replica).
+Inputs are rotated over enough copies to exceed twice the L2 size, so every
+call reads its inputs from HBM.  Extra keys report the host/device split,
+CUDA-graph replay, a padded-SDPA baseline timed the same way, the roofline
+of the attention kernel (here and on the larger B=32 / B=64 / B=512
+workloads), and the CPU oracle timed on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synthetic  # noqa: E402
+
+L2_BYTES = 126 * 1024 * 1024
+CASES = [(B, p) for B in synthetic.SERVING_BATCHES for p in synthetic.SERVING_RATES]
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
+    except Exception:
+        return 6650.0, 1590.0, "fallback"
+
+
+# --------------------------------------------------------------------------
+# clocks during the timed region
+# --------------------------------------------------------------------------
+
+class ClockSampler:
+    """nvidia-smi in a child process, sampling every 100 ms (reads only)."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu = gpu_id
+        self.proc = None
+        self.lines = []
+        self.t0 = self.t1 = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+        time.sleep(0.3)
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def mark(self, which):
+        setattr(self, which, time.time())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for ts, line in self.lines:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((ts, float(parts[1]), float(parts[2]), parts[4:]))
+            except ValueError:
+                continue
+        if not rows:
+            return None
+        inside = [r for r in rows if self.t0 is not None and self.t0 <= r[0] <= self.t1 + 0.1]
+        if not inside:
+            inside = [min(rows, key=lambda r: abs(r[0] - (self.t1 or r[0])))]
+        reasons = set()
+        names = ["active_mask", "hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in inside:
+            for name, val in zip(names[1:], r[3][1:]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r[1] for r in inside), "sm_max_mhz": max(r[2] for r in inside),
+                "reasons": sorted(reasons), "samples": len(inside)}
+
+
+# --------------------------------------------------------------------------
+# our arm
+# --------------------------------------------------------------------------
+
+def attn_bytes(w) -> int:
+    """Algorithmic bytes of one attention launch: Q, K, V read and O written
+    once, cu_seqlens read, CLS rows written."""
+    e = w.elem_bytes
+    return 4 * w.T * w.H * w.d * e + 4 * (w.B + 1) + w.B * w.H * w.d * e
+
+
+def pack_bytes(w) -> int:
+    """Algorithmic bytes of one pack launch: the mask, the kept rows read and
+    written, cu_seqlens written."""
+    return w.B * w.L_full + 2 * w.T * w.row_bytes + 4 * (w.B + 1)
+
+
+def run_ours(args, rank, world, dist):
+    import torch
+    import ragged_variable_length_b200 as rv
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    rv.load()  # fails loudly if the CUDA library is missing
+    stream = torch.cuda.current_stream()
+    hbm_peak, bf16_peak, peak_kind = peaks()
+
+    # ---- inputs: enough copies of the 12 serving batches to exceed 2x L2 ----
+    per_copy = sum(synthetic.serving(B, p).qkv.nbytes for B, p in CASES)
+    ncopies = max(2, int(np.ceil(2 * L2_BYTES / per_copy)))
+    workloads = {c: [synthetic.serving(B, p, copy=c) for B, p in CASES] for c in range(ncopies)}
+    pipes = {c: [] for c in range(ncopies)}
+    for c in range(ncopies):
+        for w in workloads[c]:
+            pl = rv.Pipeline(w.B, w.L_full, w.H, torch.float16, device=dev)
+            pl.dense_qkv.copy_(torch.from_numpy(w.qkv).to(dev))
+            pl.keep.copy_(torch.from_numpy(w.keep).to(dev))
+            pl.bind_inputs(pl.dense_qkv, pl.keep)
+            pipes[c].append(pl)
+    torch.cuda.synchronize()
+
+    def step(s):
+        for pl in pipes[s % ncopies]:
+            pl()
+            torch.cuda.synchronize()
+
+    for s in range(args.warmup):
+        step(s)
+    try:
+        sampler = ClockSampler("GPU-" + str(torch.cuda.get_device_properties(dev).uuid))
+    except Exception:
+        sampler = ClockSampler(str(dev.index))
+    sampler.start()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler.mark("t0")
+    e0.record(stream)
+    for s in range(args.steps):
+        step(s)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    sampler.mark("t1")
+    if dist:
+        dist.barrier()
+    clocks = sampler.stop()
+    ms = e0.elapsed_time(e1)
+    if dist:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    calls = args.steps * len(CASES) * world
+    us_per_call = ms * 1000.0 / calls
+
+    # ---- per-call host / device / total split, per case ----
+    detail = {}
+    reps = max(20, min(200, args.steps))
+    for i, (B, p) in enumerate(CASES):
+        host, dev_t, tot = [], [], []
+        for r in range(reps):
+            pl = pipes[r % ncopies][i]
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize()
+            t0 = time.perf_counter()
+            a.record(stream)
+            h0 = time.perf_counter()
+            pl()
+            h1 = time.perf_counter()
+            b.record(stream)
+            torch.cuda.synchronize()
+            t1 = time.perf_counter()
+            host.append((h1 - h0) * 1e6)
+            dev_t.append(a.elapsed_time(b) * 1e3)
+            tot.append((t1 - t0) * 1e6)
+        detail[f"b{B}_p{int(p * 100)}"] = {
+            "host_us": round(statistics.median(host), 2),
+            "device_us": round(statistics.median(dev_t), 2),
+            "total_us": round(statistics.median(tot), 2),
+            "total_p10_us": round(float(np.percentile(tot, 10)), 2),
+            "total_p90_us": round(float(np.percentile(tot, 90)), 2),
+        }
+
+    # ---- CUDA-graph replay: one launch per call ----
+    graph_us = None
+    try:
+        for c in range(ncopies):
+            for pl in pipes[c]:
+                pl.capture()
+        torch.cuda.synchronize()
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        g0.record(stream)
+        for s in range(args.steps):
+            for pl in pipes[s % ncopies]:
+                pl.replay()
+                torch.cuda.synchronize()
+        g1.record(stream)
+        torch.cuda.synchronize()
+        graph_us = g0.elapsed_time(g1) * 1000.0 / (args.steps * len(CASES))
+    except Exception as exc:  # capture unavailable: report, do not hide
+        graph_us = f"unavailable: {exc}"
+
+    # ---- end to end from pinned host buffers ----
+    host_in = {}
+    for c in range(ncopies):
+        for i, w in enumerate(workloads[c]):
+            host_in[(c, i)] = (torch.from_numpy(w.qkv).pin_memory(), torch.from_numpy(w.keep).pin_memory(),
+                               torch.empty((w.B, w.H, w.d), dtype=torch.float16).pin_memory())
+    h2d = sum(host_in[(0, i)][0].nbytes + host_in[(0, i)][1].nbytes for i in range(len(CASES)))
+    d2h = sum(host_in[(0, i)][2].nbytes for i in range(len(CASES)))
+
+    def e2e_step(s):
+        c = s % ncopies
+        for i, pl in enumerate(pipes[c]):
+            qkv_h, keep_h, cls_h = host_in[(c, i)]
+            pl.dense_qkv.copy_(qkv_h, non_blocking=True)
+            pl.keep.copy_(keep_h, non_blocking=True)
+            pl()
+            cls_h.copy_(pl.cls_out, non_blocking=True)
+            torch.cuda.synchronize()
+
+    for s in range(args.warmup):
+        e2e_step(s)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    x0.record(stream)
+    for s in range(args.steps):
+        e2e_step(s)
+    x1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = x0.elapsed_time(x1)
+    if dist:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_us = e2e_ms * 1000.0 / calls
+    # the last step's CLS rows must match the device result
+    ok_e2e = all(torch.equal(host_in[((args.steps - 1) % ncopies, i)][2], pl.cls_out.cpu())
+                 for i, pl in enumerate(pipes[(args.steps - 1) % ncopies]))
+
+    # ---- kernel durations: CUDA graphs of back-to-back launches, CUDA events ----
+    lib = rv.load()
+
+    def attn_launcher(pl, w):
+        D = w.H * w.d
+        base = pl.packed_qkv.data_ptr()
+        e = w.elem_bytes
+
+        def launch(strm):
+            st = lib.ragged_attn_fwd(base, base + D * e, base + 2 * D * e, 3 * D, w.d, pl.cu_seqlens.data_ptr(),
+                                     w.B, w.L_full, w.H, w.d, w.scale, 0 if w.dtype == "f16" else 1,
+                                     pl.out.data_ptr(), D, pl.cls_out.data_ptr(), strm)
+            assert st == 0, rv.ragged_last_error()
+        return launch
+
+    def pack_launcher(pl, w):
+        def launch(strm):
+            st = lib.ragged_pack(pl.dense_qkv.data_ptr(), w.B, w.L_full, w.row_bytes, pl.keep.data_ptr(),
+                                 pl.packed_qkv.data_ptr(), pl.cu_seqlens.data_ptr(), None, strm)
+            assert st == 0, rv.ragged_last_error()
+        return launch
+
+    def graph_time(launchers, replays=3):
+        """Average device time per launch of `launchers`, recorded back to back in
+        one CUDA graph and replayed between two events on the launching stream."""
+        side = torch.cuda.Stream()
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            for f in launchers:
+                f(side.cuda_stream)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=side):
+                for f in launchers:
+                    f(side.cuda_stream)
+        stream.wait_stream(side)
+        torch.cuda.synchronize()
+        g.replay()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(replays):
+            g.replay()
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / 1000.0 / (replays * len(launchers))
+
+    all_pw = [(pipes[c][i], workloads[c][i]) for c in range(ncopies) for i in range(len(CASES))]
+    t_attn = graph_time([attn_launcher(p_, w_) for p_, w_ in all_pw])
+    t_pack = graph_time([pack_launcher(p_, w_) for p_, w_ in all_pw])
+    b_attn = float(np.mean([attn_bytes(w_) for _, w_ in all_pw]))
+    b_pack = float(np.mean([pack_bytes(w_) for _, w_ in all_pw]))
+    flops = float(np.mean([w_.useful_flops() for _, w_ in all_pw]))
+    roofline = {"bound": "hbm", "achieved": round(b_attn / t_attn / 1e9, 2), "peak": hbm_peak,
+                "unit": "GB/s", "frac": round(b_attn / t_attn / 1e9 / hbm_peak, 4), "traffic": None,
+                "kernel": "attn_fwd_kernel<__half>", "avg_launch_us": round(t_attn * 1e6, 3),
+                "bytes_per_launch": int(b_attn), "launches_timed": 3 * len(all_pw), "peak_kind": peak_kind,
+                "timing": "CUDA graph of back-to-back launches over all input copies, CUDA events",
+                "useful_tflops": round(flops / t_attn / 1e12, 4),
+                "pack_kernel": {"avg_launch_us": round(t_pack * 1e6, 3), "bytes_per_launch": int(b_pack),
+                                "achieved_GBps": round(b_pack / t_pack / 1e9, 2)}}
+
+    # ---- larger workloads: attention roofline (single GPU, same kernel family) ----
+    larger = {}
+    if not args.quick:
+        for name, make, copies in (("deit_b_p80_b32", lambda c: synthetic.make_workload(
+                                        "deit_b_p80_b32", 32, 197, 12,
+                                        synthetic.deit_b_pruned80().lengths, "bf16", 1002, 1 + c), 36),
+                                   ("hires384_b64", lambda c: synthetic.hires_384(seed=1004 + 100 * c), 3),
+                                   ("sweep_b512_p0", lambda c: synthetic.sweep(0.0, seed=1005 + 100 * c), 1),
+                                   ("sweep_b512_p50", lambda c: synthetic.sweep(0.5, seed=1005 + 100 * c), 2)):
+            ws = [make(c) for c in range(copies)]
+            pls = []
+            for w in ws:
+                pl = rv.Pipeline(w.B, w.L_full, w.H, torch.float16 if w.dtype == "f16" else torch.bfloat16, device=dev)
+                pl.dense_qkv.view(torch.int16).copy_(torch.from_numpy(w.qkv.view(np.int16)).to(dev))
+                pl.keep.copy_(torch.from_numpy(w.keep).to(dev))
+                pl()
+                pls.append(pl)
+            torch.cuda.synchronize()
+            t = graph_time([attn_launcher(p_, w_) for p_, w_ in zip(pls, ws)], replays=max(3, 30 // copies))
+            bts = float(np.mean([attn_bytes(w_) for w_ in ws]))
+            fl = float(np.mean([w_.useful_flops() for w_ in ws]))
+            t_roof = max(bts / (hbm_peak * 1e9), fl / (bf16_peak * 1e12))
+            larger[name] = {"avg_launch_us": round(t * 1e6, 2), "GBps": round(bts / t / 1e9, 1),
+                            "useful_tflops": round(fl / t / 1e12, 2), "roofline_frac": round(t_roof / t, 4),
+                            "t_roof_us": round(t_roof * 1e6, 2),
+                            "l2": f"inputs rotated over {copies} copies" if copies > 1 else "packed q/k/v exceed L2"}
+            del pls
+            torch.cuda.empty_cache()
+
+    # ---- padded PyTorch SDPA baseline, same calls, same synchronisation ----
+    padded = padded_baseline(args, pipes, workloads, ncopies, stream)
+
+    # ---- CPU oracle on a bounded sample (rank 0, one GPU only) ----
+    cpu = None
+    if rank == 0 and world == 1 and not args.quick:
+        cpu = cpu_baseline(min_seconds=10.0)
+
+    gpu_launches = 2 * args.steps * len(CASES)
+    hw = {"metric": "ragged attn µs/call (host+device) at BS1-4; useful TFLOP/s & % roofline",
+          "value": round(us_per_call, 3), "unit": "µs/call", "n_gpus": world, "steps": args.steps,
+          "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 4), "higher_is_better": False,
+          "scaling": "weak", "vs_baseline": None, "dtype": "f16", "data": "synthetic",
+          "config": {"workload": "serving_deit_s_b1-4_p0-80", "B": list(synthetic.SERVING_BATCHES),
+                     "prune_rates": list(synthetic.SERVING_RATES), "jitter": 0.10, "L_full": 197,
+                     "heads": 6, "head_dim": 64, "calls_per_step": len(CASES),
+                     "call": "ragged_pipeline (pack + attention with fused CLS) + stream sync",
+                     "l2": f"inputs rotated over {ncopies} copies ({ncopies * per_copy / 2**20:.0f} MiB > 2x L2)",
+                     "parallelism": "replicas" if world > 1 else "single"},
+          "e2e": {"value": round(e2e_us, 3), "unit": "µs/call", "h2d_bytes_per_step": int(h2d),
+                  "d2h_bytes_per_step": int(d2h), "cls_matches_device": bool(ok_e2e)},
+          "gpu_launches": gpu_launches,
+          "roofline": roofline,
+          "graph_replay_us_per_call": round(graph_us, 3) if isinstance(graph_us, float) else graph_us,
+          "per_case": detail,
+          "padded_sdpa": padded,
+          "larger_workloads_attention": larger,
+          "clocks": clocks,
+          "cpu_baseline": cpu}
+    if rank == 0:
+        print(json.dumps(hw), flush=True)
+
+
+def padded_baseline(args, pipes, workloads, ncopies, stream):
+    """Pad every survivor set to the batch's longest (Lmax known on the host),
+    mask padded keys, run torch SDPA, take the CLS rows."""
+    import torch
+    import torch.nn.functional as F
+
+    def call(pl, Lmax):
+        keep = pl.keep.bool()
+        keep[:, 0] = True
+        L = keep.sum(1)
+        idx = torch.argsort((~keep).to(torch.int8), dim=1, stable=True)[:, :Lmax]
+        B, _, three, H, d = pl.dense_qkv.shape
+        g = torch.gather(pl.dense_qkv, 1, idx[:, :, None, None, None].expand(B, Lmax, three, H, d))
+        q, k, v = g.permute(2, 0, 3, 1, 4).unbind(0)             # [B, H, Lmax, d]
+        valid = torch.arange(Lmax, device=keep.device)[None, :] < L[:, None]
+        o = F.scaled_dot_product_attention(q, k, v, attn_mask=valid[:, None, None, :])
+        return o[:, :, 0]
+
+    res = {}
+    reps = max(20, min(200, args.steps))
+    for i, (B, p) in enumerate(CASES):
+        tot = []
+        for r in range(reps + 3):
+            c = r % ncopies
+            Lmax = int(workloads[c][i].Lmax)
+            torch.cuda.synchronize()
+            t0 = time.perf_counter()
+            cls = call(pipes[c][i], Lmax)
+            torch.cuda.synchronize()
+            if r >= 3:
+                tot.append((time.perf_counter() - t0) * 1e6)
+        ref = pipes[0][i].cls_out.float()
+        err = float((call(pipes[0][i], int(workloads[0][i].Lmax)).float() - ref).abs().max())
+        res[f"b{B}_p{int(p * 100)}"] = {"total_us": round(statistics.median(tot), 2), "max_abs_vs_ragged": err}
+    return res
+
+
+def cpu_baseline(min_seconds=10.0):
+    """The CPU oracle, as it stands, on the bench's calls (whole pipeline per call)."""
+    import oracle
+    ws = [synthetic.serving(B, p) for B, p in CASES]
+    oracle.pipeline(ws[0])
+    n, t0 = 0, time.perf_counter()
+    while True:
+        for w in ws:
+            oracle.pipeline(w)
+            n += 1
+        if time.perf_counter() - t0 >= min_seconds:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": round(dt * 1e6 / n, 1), "unit": "µs/call", "cores": oracle.num_cores(), "kind": "oracle",
+            "sample": f"{n} calls ({n // len(ws)} passes over the 12 serving batches), fp64 C oracle, "
+                      f"{oracle.num_cores()} threads"}
+
+
+# --------------------------------------------------------------------------
+# reference arm: the CPU oracle on the same workload
+# --------------------------------------------------------------------------
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    import oracle
+    ws = [synthetic.serving(B, p) for B, p in CASES]
+    for s in range(args.warmup):
+        oracle.pipeline(ws[s % len(ws)])
+    n, t0 = 0, time.perf_counter()
+    for s in range(args.steps):
+        for w in ws:
+            oracle.pipeline(w)
+            n += 1
+    dt = time.perf_counter() - t0
+    v = dt * 1e6 / n
+    cores = oracle.num_cores()
+    print(json.dumps({
+        "impl": "reference", "metric": "ragged attn µs/call (host+device) at BS1-4; useful TFLOP/s & % roofline",
+        "value": round(v, 1), "unit": "µs/call", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(dt * 1000 / args.steps, 3), "higher_is_better": False, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "serving_deit_s_b1-4_p0-80", "B": list(synthetic.SERVING_BATCHES),
+                   "prune_rates": list(synthetic.SERVING_RATES), "L_full": 197, "heads": 6, "head_dim": 64,
+                   "calls_per_step": len(CASES), "call": "CPU oracle pipeline (pack, attention, CLS)"},
+        "cpu_baseline": {"value": round(v, 1), "unit": "µs/call", "cores": cores, "kind": "oracle",
+                         "sample": f"{args.steps} steps x {len(ws)} calls, fp64 C oracle, {cores} threads"},
+        "e2e": {"value": round(v, 1), "unit": "µs/call", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--quick", action="store_true", help="skip the larger workloads and the CPU baseline")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    dist = None
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as tdist
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        dist = tdist
+    try:
+        run_ours(args, rank, world, dist)
+    finally:
+        if dist:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

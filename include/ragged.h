@@ -1,0 +1,202 @@
+/*
+ * ragged.h - C ABI of the pack -> attend -> unpack pipeline for token-pruned
+ * Vision Transformers, after "Dispatch-Aware Ragged Attention for Pruned
+ * Vision Transformers" (arXiv 2604.15408).
+ *
+ * The pipeline has three steps:
+ *   1. pack:   per-image keep masks -> cu_seqlens, and the surviving token
+ *              rows (CLS always kept) gathered into one flat ragged buffer;
+ *   2. attend: bidirectional multi-head softmax attention over every
+ *              variable-length sequence of that buffer, with no causal mask,
+ *              no KV cache and no padding;
+ *   3. unpack: extract each sequence's CLS row, or scatter rows back to their
+ *              dense positions.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Pointers named as device buffers are device memory of the current CUDA
+ *    device, owned by the caller.  The library allocates nothing per call and
+ *    keeps no pointer after returning.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ *    stream).  Work is only enqueued: no call synchronises with the device,
+ *    except ragged_get_device_status, which says so.
+ *  - Every call returns a ragged_status.  Argument errors are detected on the
+ *    host before anything is enqueued; nothing is launched then and
+ *    ragged_last_error() describes the problem.  A launch failure reported by
+ *    the CUDA runtime returns RAGGED_ERR_CUDA.  Problems only the device can
+ *    see (inconsistent cu_seqlens, a bounded wait that gave up) set bits of a
+ *    per-device status word read by ragged_get_device_status; the affected
+ *    sequence is skipped rather than read or written out of bounds.
+ *  - Calls may be captured into a CUDA graph; none of them synchronises or
+ *    allocates.
+ *  - Sizes are int64_t; lengths and offsets inside cu_seqlens are int32, so
+ *    B * L_full must stay below 2^31.
+ */
+#ifndef RAGGED_H
+#define RAGGED_H
+
+#include <stdint.h>
+
+/* Exported symbols (the library is built with hidden default visibility). */
+#if defined(RAGGED_BUILD) && defined(__GNUC__)
+#define RAGGED_API __attribute__((visibility("default")))
+#else
+#define RAGGED_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum ragged_status {
+    RAGGED_OK = 0,
+    RAGGED_ERR_INVALID_ARG = 1, /* null pointer, negative size, misalignment, ... */
+    RAGGED_ERR_UNSUPPORTED = 2, /* valid request outside what is implemented    */
+    RAGGED_ERR_CUDA = 3,        /* the CUDA runtime reported an error           */
+    RAGGED_ERR_DEVICE = 4       /* reserved for device-side failures            */
+} ragged_status;
+
+typedef enum ragged_dtype {
+    RAGGED_F16 = 0,  /* IEEE binary16                     */
+    RAGGED_BF16 = 1, /* bfloat16                          */
+    RAGGED_F32 = 2   /* IEEE binary32 (FFMA check path)   */
+} ragged_dtype;
+
+/* Bits of the per-device status word (ragged_get_device_status). */
+#define RAGGED_DEV_BAD_SEQLENS 0x1u /* cu_seqlens decreasing, or a length > max_seqlen */
+#define RAGGED_DEV_TIMEOUT 0x2u     /* a bounded device-side wait gave up              */
+
+/* Largest L_full accepted by pack/unpack and max_seqlen by attention. */
+#define RAGGED_MAX_TOKENS 16384
+
+/*
+ * ragged_pack - survivor bookkeeping and gather (step 1).
+ * Paper: radpulse article, section "Integrated pack pipeline, 2.24x
+ * end-to-end" (cu_seqlens computed first, survivors copied with coalesced
+ * copies into a contiguous flat tensor) and its section on the FA2 dispatch
+ * ceiling (survivors packed into a contiguous ragged buffer for a varlen API).
+ *
+ *   dense       device, [B, L_full] rows of row_bytes bytes, contiguous,
+ *               16-byte aligned.  Read only.
+ *   B, L_full   images and dense tokens per image; B >= 0, 1 <= L_full <=
+ *               RAGGED_MAX_TOKENS.
+ *   row_bytes   bytes per token row; a positive multiple of 16.
+ *   keep        device, uint8 [B, L_full], any alignment.  Nonzero keeps the
+ *               token.  Token 0 (CLS) is kept whatever keep[b, 0] says.
+ *   packed      device, capacity B * L_full rows of row_bytes, 16-byte
+ *               aligned.  On completion rows 0..T-1 hold the survivors, image
+ *               by image, each image's survivors in ascending token order
+ *               (so CLS of image b is row cu_seqlens[b]).  Rows >= T are not
+ *               written.
+ *   cu_seqlens  device, int32 [B + 1]: cu[0] = 0, cu[b+1] = cu[b] + L_b where
+ *               L_b >= 1 is the survivor count of image b; T = cu[B].
+ *   src_idx     device int32 [B * L_full] or NULL: for each packed row t,
+ *               the flat dense row b * L_full + j it was copied from.
+ * B == 0 writes cu_seqlens[0] = 0 and nothing else.
+ */
+RAGGED_API ragged_status ragged_pack(const void *dense, int64_t B, int64_t L_full, int64_t row_bytes,
+                          const uint8_t *keep, void *packed, int32_t *cu_seqlens,
+                          int32_t *src_idx, void *stream);
+
+/*
+ * ragged_attn_fwd - ragged bidirectional attention (step 2).
+ * Paper: abstract (lightweight bidirectional attention kernel over ragged
+ * ViT sequences) and radpulse section "Bypassing the binding" (no causal
+ * mask, no KV cache, no softmax_lse workspace).  For every sequence b (rows
+ * cu[b] .. cu[b+1]-1) and head h:
+ *        O_b,h = softmax(scale * Q_b,h K_b,h^T) V_b,h
+ * over the L_b rows of that sequence only.  Accumulation and softmax are in
+ * fp32; the output is rounded to nearest even in the input format.
+ *
+ *   q, k, v        device; element (t, h, c) of each is at
+ *                  base[t * tok_stride + h * head_stride + c].  Separate
+ *                  tensors or the three slices of one fused [T, 3, H, 64]
+ *                  buffer.  16-byte aligned.
+ *   tok_stride, head_stride   in elements; each times the element size must
+ *                  be a multiple of 16 bytes.
+ *   cu_seqlens     device int32 [B + 1], non-decreasing, cu[0] = 0 (as
+ *                  written by ragged_pack).  Read on the device only.
+ *   B              number of sequences, >= 0 (0 is a no-op).
+ *   max_seqlen     host-side upper bound on every L_b (e.g. L_full), 1 ..
+ *                  RAGGED_MAX_TOKENS.  Sizes the launch; a sequence longer
+ *                  than this is skipped and RAGGED_DEV_BAD_SEQLENS is set.
+ *   H, head_dim    heads (>= 1) and head dimension (only 64 is implemented:
+ *                  other values return RAGGED_ERR_UNSUPPORTED).
+ *   scale          softmax scale, positive and finite; usually 1/sqrt(head_dim).
+ *   dtype          format of q, k, v, out and cls_out.
+ *   out            device, element (t, h, c) at out[t * out_tok_stride + h *
+ *                  head_dim + c]; out_tok_stride >= H * head_dim, times the
+ *                  element size a multiple of 16 bytes.  16-byte aligned.
+ *   cls_out        device [B, H * head_dim] contiguous, or NULL: receives
+ *                  row cu[b] of out for every b (the CLS extraction of step
+ *                  3 fused into the attention epilogue).
+ */
+RAGGED_API ragged_status ragged_attn_fwd(const void *q, const void *k, const void *v, int64_t tok_stride,
+                              int64_t head_stride, const int32_t *cu_seqlens, int64_t B,
+                              int64_t max_seqlen, int64_t H, int64_t head_dim, float scale,
+                              ragged_dtype dtype, void *out, int64_t out_tok_stride,
+                              void *cls_out, void *stream);
+
+/*
+ * ragged_unpack_cls - CLS extraction (step 3).
+ * Paper: radpulse section "Integrated pack pipeline" (after attention and the
+ * MLP run on the packed tokens, the CLS token is extracted).
+ *
+ *   packed      device, rows of row_bytes, contiguous, 16-byte aligned.
+ *   cu_seqlens  device int32 [B + 1].
+ *   row_bytes   positive multiple of 16.
+ *   cls_out     device [B] rows of row_bytes: cls_out[b] = packed[cu[b]].
+ */
+RAGGED_API ragged_status ragged_unpack_cls(const void *packed, const int32_t *cu_seqlens, int64_t B,
+                                int64_t row_bytes, void *cls_out, void *stream);
+
+/*
+ * ragged_unpack - scatter back (step 3, full form).
+ * The inverse of ragged_pack's gather: dense_out[b, j] = packed[cu[b] + r]
+ * for the r-th survivor j of image b (same keep mask, CLS always kept).  Rows
+ * of dropped tokens are left untouched.
+ *
+ *   packed      device, rows of row_bytes, 16-byte aligned.
+ *   cu_seqlens  device int32 [B + 1] from ragged_pack on the same keep mask.
+ *   keep        device uint8 [B, L_full].
+ *   dense_out   device [B, L_full] rows of row_bytes, 16-byte aligned.
+ */
+RAGGED_API ragged_status ragged_unpack(const void *packed, const int32_t *cu_seqlens, const uint8_t *keep,
+                            int64_t B, int64_t L_full, int64_t row_bytes, void *dense_out,
+                            void *stream);
+
+/*
+ * ragged_pipeline - pack -> attend -> CLS in one host call (two launches).
+ * dense_qkv is one fused [B, L_full, 3, H, head_dim] buffer (q, k, v along
+ * the third axis); it is packed into packed_qkv [B * L_full, 3, H, head_dim]
+ * (capacity), attention reads the packed rows, and writes out [T, H,
+ * head_dim] (capacity B * L_full rows) and, if cls_out is not NULL, cls_out
+ * [B, H * head_dim].  Requirements as for ragged_pack and ragged_attn_fwd,
+ * with max_seqlen = L_full.
+ */
+RAGGED_API ragged_status ragged_pipeline(const void *dense_qkv, const uint8_t *keep, int64_t B,
+                              int64_t L_full, int64_t H, int64_t head_dim, float scale,
+                              ragged_dtype dtype, void *packed_qkv, int32_t *cu_seqlens,
+                              void *out, void *cls_out, void *stream);
+
+/*
+ * ragged_get_device_status - read and clear the status word of the current
+ * device.  Synchronises with `stream` (the only call that does).  *host_out
+ * receives the RAGGED_DEV_* bits set since the previous read.
+ */
+RAGGED_API ragged_status ragged_get_device_status(uint32_t *host_out, void *stream);
+
+/* Static description of a status code. */
+RAGGED_API const char *ragged_status_string(ragged_status status);
+
+/* Description of the last error returned on the calling host thread. */
+RAGGED_API const char *ragged_last_error(void);
+
+/* ABI version of the library (bumped when a signature changes). */
+RAGGED_API int32_t ragged_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RAGGED_H */

@@ -1,0 +1,70 @@
+"""Builds libragged.so (the CUDA kernels and their C ABI) for sm_100a with nvcc.
+
+    python -m ragged_variable_length_b200.build [--force] [--verbose-ptxas]
+
+The library is built in-tree, next to this file, and statically links the
+CUDA runtime so that it does not depend on which libcudart the process loads.
+"""
+from __future__ import annotations
+
+import glob
+import os
+import shutil
+import subprocess
+import sys
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(HERE)
+CSRC = os.path.join(HERE, "csrc")
+INCLUDE = os.path.join(ROOT, "include")
+LIB = os.path.join(HERE, "libragged.so")
+MAIN = os.path.join(CSRC, "ragged_api.cu")
+
+ARCH_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a"]
+
+
+def nvcc() -> str:
+    for cand in (os.environ.get("NVCC"), shutil.which("nvcc"), "/usr/local/cuda/bin/nvcc"):
+        if cand and os.path.exists(cand):
+            return cand
+    raise RuntimeError("nvcc not found")
+
+
+def sources() -> list:
+    return sorted(glob.glob(os.path.join(CSRC, "*.cu")) + glob.glob(os.path.join(CSRC, "*.cuh")) +
+                  glob.glob(os.path.join(INCLUDE, "*.h")))
+
+
+def stale() -> bool:
+    if not os.path.exists(LIB):
+        return True
+    t = os.path.getmtime(LIB)
+    return any(os.path.getmtime(s) > t for s in sources())
+
+
+def command(out: str, ptxas_verbose: bool = False) -> list:
+    cmd = [nvcc(), *ARCH_FLAGS, "-O3", "-lineinfo", "-std=c++17", "-shared", "-Xcompiler", "-fPIC",
+           "-Xcompiler", "-fvisibility=hidden", "--expt-relaxed-constexpr", "-cudart", "static",
+           f"-I{INCLUDE}", f"-I{CSRC}", "-DRAGGED_BUILD", MAIN, "-o", out]
+    if ptxas_verbose:
+        cmd[1:1] = ["-Xptxas", "-v"]
+    return cmd
+
+
+def build(force: bool = False, ptxas_verbose: bool = False) -> str:
+    if not force and not stale():
+        return LIB
+    tmp = f"{LIB}.{os.getpid()}.tmp"
+    proc = subprocess.run(command(tmp, ptxas_verbose), capture_output=True, text=True)
+    if proc.returncode != 0:
+        sys.stderr.write(proc.stdout + proc.stderr)
+        raise RuntimeError("nvcc failed building libragged.so")
+    if ptxas_verbose:
+        sys.stderr.write(proc.stdout + proc.stderr)
+    os.replace(tmp, LIB)
+    return LIB
+
+
+if __name__ == "__main__":
+    build(force="--force" in sys.argv, ptxas_verbose="--verbose-ptxas" in sys.argv)
+    print(LIB)

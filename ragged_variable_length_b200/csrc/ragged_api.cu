@@ -1,0 +1,284 @@
+// C ABI of the ragged pack -> attend -> unpack library (declared in ragged.h).
+//
+// The host side of every call is a handful of integer checks followed by one
+// kernel launch: no allocation, no synchronisation, no per-call workspace
+// (the paper's radpulse section "Bypassing the binding" locates the
+// dispatch floor of FA2's varlen path in argument conversion, output and
+// softmax_lse allocation and the launch itself).
+#include <cstdarg>
+#include <cstdio>
+#include <type_traits>
+
+#include "attn_f32.cuh"
+#include "attn_mma.cuh"
+#include "common.cuh"
+#include "pack.cuh"
+
+namespace {
+
+constexpr int32_t kAbiVersion = 1;
+constexpr int kMaxDevices = 64;
+// Shared memory of the pack / unpack survivor list at the largest L_full.
+constexpr int kMaxListBytes = RAGGED_MAX_TOKENS * static_cast<int>(sizeof(int));
+
+thread_local char g_last_error[256] = "";
+
+ragged_status fail(ragged_status s, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_last_error, sizeof g_last_error, fmt, ap);
+    va_end(ap);
+    return s;
+}
+
+ragged_status cuda_check(cudaError_t e, const char* what) {
+    if (e == cudaSuccess) return RAGGED_OK;
+    return fail(RAGGED_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Multiprocessor count of the current device, cached per device.
+int sm_count() {
+    static int cache[kMaxDevices] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+    if (cache[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        cache[dev] = n;
+    }
+    return cache[dev];
+}
+
+// Opt-in shared-memory sizes are set once per device and kernel.
+template <typename Kernel>
+ragged_status ensure_smem(Kernel kernel, int bytes, bool (&done)[kMaxDevices]) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+        return fail(RAGGED_ERR_CUDA, "cudaGetDevice failed");
+    if (!done[dev]) {
+        ragged_status s = cuda_check(
+            cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes),
+            "cudaFuncSetAttribute");
+        if (s != RAGGED_OK) return s;
+        done[dev] = true;
+    }
+    return RAGGED_OK;
+}
+
+ragged_status check_rows(int64_t B, int64_t L_full, int64_t row_bytes) {
+    if (B < 0) return fail(RAGGED_ERR_INVALID_ARG, "B = %lld is negative", (long long)B);
+    if (B > 65535) return fail(RAGGED_ERR_UNSUPPORTED, "B = %lld exceeds 65535", (long long)B);
+    if (L_full < 1 || L_full > RAGGED_MAX_TOKENS)
+        return fail(RAGGED_ERR_INVALID_ARG, "L_full = %lld outside [1, %d]", (long long)L_full,
+                    RAGGED_MAX_TOKENS);
+    if (B * L_full >= (int64_t(1) << 31))
+        return fail(RAGGED_ERR_UNSUPPORTED, "B * L_full = %lld does not fit int32 offsets",
+                    (long long)(B * L_full));
+    if (row_bytes <= 0 || row_bytes % 16 != 0)
+        return fail(RAGGED_ERR_INVALID_ARG, "row_bytes = %lld must be a positive multiple of 16",
+                    (long long)row_bytes);
+    if (L_full * (row_bytes / 16) >= (int64_t(1) << 31))
+        return fail(RAGGED_ERR_UNSUPPORTED, "rows of %lld bytes are too long", (long long)row_bytes);
+    return RAGGED_OK;
+}
+
+// Row splits per image: enough CTAs to cover every SM a few times, but at
+// least eight rows per CTA on average.
+int pack_splits(int64_t B, int64_t L_full) {
+    const int64_t target = 4LL * sm_count();
+    int64_t s = (target + B - 1) / B;
+    const int64_t cap = (L_full + 7) / 8;
+    if (s > cap) s = cap;
+    if (s < 1) s = 1;
+    if (s > 65535) s = 65535;
+    return static_cast<int>(s);
+}
+
+bool g_pack_smem[kMaxDevices], g_unpack_smem[kMaxDevices];
+bool g_mma_f16_smem[kMaxDevices], g_mma_bf16_smem[kMaxDevices], g_f32_smem[kMaxDevices];
+
+}  // namespace
+
+extern "C" {
+
+int32_t ragged_abi_version(void) { return kAbiVersion; }
+
+const char* ragged_last_error(void) { return g_last_error; }
+
+const char* ragged_status_string(ragged_status s) {
+    switch (s) {
+        case RAGGED_OK: return "ok";
+        case RAGGED_ERR_INVALID_ARG: return "invalid argument";
+        case RAGGED_ERR_UNSUPPORTED: return "unsupported";
+        case RAGGED_ERR_CUDA: return "CUDA runtime error";
+        case RAGGED_ERR_DEVICE: return "device-side error";
+    }
+    return "unknown status";
+}
+
+ragged_status ragged_pack(const void* dense, int64_t B, int64_t L_full, int64_t row_bytes,
+                          const uint8_t* keep, void* packed, int32_t* cu_seqlens,
+                          int32_t* src_idx, void* stream) {
+    ragged_status st = check_rows(B, L_full, row_bytes);
+    if (st != RAGGED_OK) return st;
+    if (cu_seqlens == nullptr) return fail(RAGGED_ERR_INVALID_ARG, "cu_seqlens is NULL");
+    if ((reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) || (reinterpret_cast<uintptr_t>(src_idx) & 3u))
+        return fail(RAGGED_ERR_INVALID_ARG, "cu_seqlens / src_idx must be 4-byte aligned");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (B == 0) return cuda_check(cudaMemsetAsync(cu_seqlens, 0, sizeof(int32_t), s), "cudaMemsetAsync");
+    if (dense == nullptr || keep == nullptr || packed == nullptr)
+        return fail(RAGGED_ERR_INVALID_ARG, "dense, keep and packed must not be NULL");
+    if (!aligned16(dense) || !aligned16(packed))
+        return fail(RAGGED_ERR_INVALID_ARG, "dense and packed must be 16-byte aligned");
+    const int smem = static_cast<int>(L_full * sizeof(int));
+    st = ensure_smem(ragged::pack_kernel, kMaxListBytes, g_pack_smem);
+    if (st != RAGGED_OK) return st;
+    const dim3 grid(pack_splits(B, L_full), static_cast<unsigned>(B));
+    ragged::pack_kernel<<<grid, ragged::kPackThreads, smem, s>>>(
+        static_cast<const uint4*>(dense), static_cast<int>(L_full),
+        static_cast<uint32_t>(row_bytes / 16), keep, static_cast<uint4*>(packed), cu_seqlens, src_idx);
+    return cuda_check(cudaGetLastError(), "pack launch");
+}
+
+ragged_status ragged_unpack(const void* packed, const int32_t* cu_seqlens, const uint8_t* keep,
+                            int64_t B, int64_t L_full, int64_t row_bytes, void* dense_out,
+                            void* stream) {
+    ragged_status st = check_rows(B, L_full, row_bytes);
+    if (st != RAGGED_OK) return st;
+    if (B == 0) return RAGGED_OK;
+    if (packed == nullptr || cu_seqlens == nullptr || keep == nullptr || dense_out == nullptr)
+        return fail(RAGGED_ERR_INVALID_ARG, "packed, cu_seqlens, keep and dense_out must not be NULL");
+    if (!aligned16(packed) || !aligned16(dense_out) || (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u))
+        return fail(RAGGED_ERR_INVALID_ARG, "packed / dense_out must be 16-byte aligned, cu_seqlens 4-byte");
+    const int smem = static_cast<int>(L_full * sizeof(int));
+    st = ensure_smem(ragged::unpack_kernel, kMaxListBytes, g_unpack_smem);
+    if (st != RAGGED_OK) return st;
+    const dim3 grid(pack_splits(B, L_full), static_cast<unsigned>(B));
+    ragged::unpack_kernel<<<grid, ragged::kPackThreads, smem, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<const uint4*>(packed), cu_seqlens, static_cast<int>(L_full),
+        static_cast<uint32_t>(row_bytes / 16), keep, static_cast<uint4*>(dense_out));
+    return cuda_check(cudaGetLastError(), "unpack launch");
+}
+
+ragged_status ragged_unpack_cls(const void* packed, const int32_t* cu_seqlens, int64_t B,
+                                int64_t row_bytes, void* cls_out, void* stream) {
+    if (B < 0) return fail(RAGGED_ERR_INVALID_ARG, "B = %lld is negative", (long long)B);
+    if (row_bytes <= 0 || row_bytes % 16 != 0)
+        return fail(RAGGED_ERR_INVALID_ARG, "row_bytes = %lld must be a positive multiple of 16",
+                    (long long)row_bytes);
+    if (B == 0) return RAGGED_OK;
+    if (packed == nullptr || cu_seqlens == nullptr || cls_out == nullptr)
+        return fail(RAGGED_ERR_INVALID_ARG, "packed, cu_seqlens and cls_out must not be NULL");
+    if (!aligned16(packed) || !aligned16(cls_out) || (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u))
+        return fail(RAGGED_ERR_INVALID_ARG, "packed / cls_out must be 16-byte aligned, cu_seqlens 4-byte");
+    const int64_t n = B * (row_bytes / 16);
+    if (B > (int64_t(1) << 31) || n >= (int64_t(1) << 40))
+        return fail(RAGGED_ERR_UNSUPPORTED, "CLS extraction too large");
+    const int64_t blocks = (n + 255) / 256;
+    ragged::unpack_cls_kernel<<<static_cast<unsigned>(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<const uint4*>(packed), cu_seqlens, static_cast<int>(B),
+        static_cast<uint32_t>(row_bytes / 16), static_cast<uint4*>(cls_out));
+    return cuda_check(cudaGetLastError(), "unpack_cls launch");
+}
+
+ragged_status ragged_attn_fwd(const void* q, const void* k, const void* v, int64_t tok_stride,
+                              int64_t head_stride, const int32_t* cu_seqlens, int64_t B,
+                              int64_t max_seqlen, int64_t H, int64_t head_dim, float scale,
+                              ragged_dtype dtype, void* out, int64_t out_tok_stride,
+                              void* cls_out, void* stream) {
+    if (B < 0) return fail(RAGGED_ERR_INVALID_ARG, "B = %lld is negative", (long long)B);
+    if (B > 65535) return fail(RAGGED_ERR_UNSUPPORTED, "B = %lld exceeds 65535", (long long)B);
+    if (dtype != RAGGED_F16 && dtype != RAGGED_BF16 && dtype != RAGGED_F32)
+        return fail(RAGGED_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
+    if (head_dim != 64) return fail(RAGGED_ERR_UNSUPPORTED, "head_dim = %lld (only 64 is implemented)", (long long)head_dim);
+    if (H < 1 || H > 65535) return fail(RAGGED_ERR_INVALID_ARG, "H = %lld outside [1, 65535]", (long long)H);
+    if (max_seqlen < 1 || max_seqlen > RAGGED_MAX_TOKENS)
+        return fail(RAGGED_ERR_INVALID_ARG, "max_seqlen = %lld outside [1, %d]", (long long)max_seqlen,
+                    RAGGED_MAX_TOKENS);
+    if (!(scale > 0.f) || scale > 3.0e38f)
+        return fail(RAGGED_ERR_INVALID_ARG, "scale must be a positive finite number");
+    if (B == 0) return RAGGED_OK;
+    if (!q || !k || !v || !out || !cu_seqlens)
+        return fail(RAGGED_ERR_INVALID_ARG, "q, k, v, out and cu_seqlens must not be NULL");
+    const int64_t esz = dtype == RAGGED_F32 ? 4 : 2;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(cls_out) ||
+        (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u))
+        return fail(RAGGED_ERR_INVALID_ARG, "q, k, v, out, cls_out must be 16-byte aligned");
+    if (tok_stride <= 0 || head_stride < 0 || (tok_stride * esz) % 16 || (head_stride * esz) % 16)
+        return fail(RAGGED_ERR_INVALID_ARG, "tok_stride / head_stride must be multiples of 16 bytes");
+    if (out_tok_stride < H * head_dim || (out_tok_stride * esz) % 16)
+        return fail(RAGGED_ERR_INVALID_ARG, "out_tok_stride must be >= H * head_dim and a multiple of 16 bytes");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    ragged_status st;
+    if (dtype == RAGGED_F32) {
+        using namespace ragged::f32_attn;
+        st = ensure_smem(attn_fwd_f32_kernel, kSmemBytes, g_f32_smem);
+        if (st != RAGGED_OK) return st;
+        const dim3 grid(static_cast<unsigned>((max_seqlen + kBlockM - 1) / kBlockM), static_cast<unsigned>(H),
+                        static_cast<unsigned>(B));
+        attn_fwd_f32_kernel<<<grid, kThreads, kSmemBytes, s>>>(
+            static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v),
+            tok_stride, head_stride, cu_seqlens, static_cast<int>(max_seqlen), static_cast<int>(H), scale,
+            static_cast<float*>(out), out_tok_stride, static_cast<float*>(cls_out));
+        return cuda_check(cudaGetLastError(), "attention (f32) launch");
+    }
+    using namespace ragged::mma_attn;
+    const dim3 grid(static_cast<unsigned>((max_seqlen + kBlockM - 1) / kBlockM), static_cast<unsigned>(H),
+                    static_cast<unsigned>(B));
+    const float scale_log2 = scale * 1.4426950408889634f;
+    if (dtype == RAGGED_F16) {
+        st = ensure_smem(attn_fwd_kernel<__half>, kSmemBytes, g_mma_f16_smem);
+        if (st != RAGGED_OK) return st;
+        attn_fwd_kernel<__half><<<grid, kThreads, kSmemBytes, s>>>(
+            static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(k), static_cast<const uint16_t*>(v),
+            tok_stride, head_stride, cu_seqlens, static_cast<int>(max_seqlen), static_cast<int>(H),
+            scale_log2, static_cast<uint16_t*>(out), out_tok_stride, static_cast<uint16_t*>(cls_out));
+    } else {
+        st = ensure_smem(attn_fwd_kernel<__nv_bfloat16>, kSmemBytes, g_mma_bf16_smem);
+        if (st != RAGGED_OK) return st;
+        attn_fwd_kernel<__nv_bfloat16><<<grid, kThreads, kSmemBytes, s>>>(
+            static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(k), static_cast<const uint16_t*>(v),
+            tok_stride, head_stride, cu_seqlens, static_cast<int>(max_seqlen), static_cast<int>(H),
+            scale_log2, static_cast<uint16_t*>(out), out_tok_stride, static_cast<uint16_t*>(cls_out));
+    }
+    return cuda_check(cudaGetLastError(), "attention launch");
+}
+
+ragged_status ragged_pipeline(const void* dense_qkv, const uint8_t* keep, int64_t B, int64_t L_full,
+                              int64_t H, int64_t head_dim, float scale, ragged_dtype dtype,
+                              void* packed_qkv, int32_t* cu_seqlens, void* out, void* cls_out,
+                              void* stream) {
+    if (head_dim != 64) return fail(RAGGED_ERR_UNSUPPORTED, "head_dim = %lld (only 64 is implemented)", (long long)head_dim);
+    if (H < 1 || H > 65535) return fail(RAGGED_ERR_INVALID_ARG, "H = %lld outside [1, 65535]", (long long)H);
+    if (dtype != RAGGED_F16 && dtype != RAGGED_BF16 && dtype != RAGGED_F32)
+        return fail(RAGGED_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
+    const int64_t esz = dtype == RAGGED_F32 ? 4 : 2;
+    const int64_t D = H * head_dim;
+    ragged_status st = ragged_pack(dense_qkv, B, L_full, 3 * D * esz, keep, packed_qkv, cu_seqlens,
+                                   nullptr, stream);
+    if (st != RAGGED_OK || B == 0) return st;
+    const char* base = static_cast<const char*>(packed_qkv);
+    return ragged_attn_fwd(base, base + D * esz, base + 2 * D * esz, 3 * D, head_dim, cu_seqlens, B,
+                           L_full, H, head_dim, scale, dtype, out, D, cls_out, stream);
+}
+
+ragged_status ragged_get_device_status(uint32_t* host_out, void* stream) {
+    if (host_out == nullptr) return fail(RAGGED_ERR_INVALID_ARG, "host_out is NULL");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    unsigned int value = 0, zero = 0;
+    ragged_status st = cuda_check(
+        cudaMemcpyFromSymbolAsync(&value, ragged::g_dev_status, sizeof value, 0, cudaMemcpyDeviceToHost, s),
+        "reading the device status word");
+    if (st != RAGGED_OK) return st;
+    st = cuda_check(cudaMemcpyToSymbolAsync(ragged::g_dev_status, &zero, sizeof zero, 0, cudaMemcpyHostToDevice, s),
+                    "clearing the device status word");
+    if (st != RAGGED_OK) return st;
+    st = cuda_check(cudaStreamSynchronize(s), "cudaStreamSynchronize");
+    if (st != RAGGED_OK) return st;
+    *host_out = value;
+    return RAGGED_OK;
+}
+
+}  // extern "C"

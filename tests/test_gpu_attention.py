@@ -1,0 +1,168 @@
+"""GPU parity of ragged attention against the fp64 CPU oracle, through the C ABI.
+
+Bar: max-abs error <= 4e-3 for f16 / bf16 inputs (fp32 accumulation, output
+rounded to the input format), and max |gpu - oracle| <= 1e-5 max |oracle| on
+the fp32 check path.  Small cases are compared element by element; the full
+workloads are compared on sampled sequences (always including the shortest
+and the longest), in the same launch configuration the benchmark times.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import ragged_variable_length_b200 as rv
+import synthetic
+from helpers import TORCH_DTYPE, attn_error, to_device, to_f64
+
+pytestmark = pytest.mark.gpu
+
+
+def run_pipeline(w, separate_qkv=False, out_pad=0):
+    """Device pack -> attend (with fused CLS) for a synthetic workload."""
+    dense = to_device(w.qkv, w.dtype)
+    keep = torch.from_numpy(w.keep).cuda()
+    packed, cu = rv.ragged_pack(dense, keep)
+    T_cap = w.B * w.L_full
+    out_full = torch.full((T_cap, w.H * w.d + out_pad), float("nan"), dtype=TORCH_DTYPE[w.dtype], device="cuda")
+    out = out_full[:, :w.H * w.d].view(T_cap, w.H, w.d) if out_pad == 0 else \
+        out_full.as_strided((T_cap, w.H, w.d), (w.H * w.d + out_pad, w.d, 1))
+    cls = torch.full((w.B, w.H, w.d), float("nan"), dtype=TORCH_DTYPE[w.dtype], device="cuda")
+    if separate_qkv:
+        q, k, v = (packed[:, i].contiguous() for i in range(3))
+    else:
+        q, k, v = packed[:, 0], packed[:, 1], packed[:, 2]
+    rv.ragged_attn_fwd(q, k, v, cu, w.L_full, w.scale, out=out, cls_out=cls)
+    torch.cuda.synchronize()
+    assert rv.ragged_get_device_status() == 0
+    return cu.cpu().numpy(), out, cls, out_full
+
+
+def sample_sequences(lengths, n, seed=0):
+    L = np.asarray(lengths)
+    pick = {int(np.argmin(L)), int(np.argmax(L))}
+    rng = np.random.default_rng(seed)
+    while len(pick) < min(n, len(L)):
+        pick.add(int(rng.integers(0, len(L))))
+    return sorted(pick)
+
+
+def check_against_oracle(w, seqs=None, **kw):
+    cu, out, cls, out_full = run_pipeline(w, **kw)
+    packed_o, cu_o = oracle.pack(w.qkv, w.keep)
+    assert np.array_equal(cu, cu_o)
+    ref = oracle.attention(packed_o[:, 0], packed_o[:, 1], packed_o[:, 2], cu_o, w.dtype, w.scale, seqs=seqs)
+    T = int(cu[-1])
+    got = to_f64(out[:T])
+    rows = np.concatenate([np.arange(cu[b], cu[b + 1]) for b in (seqs if seqs is not None else range(w.B))])
+    err, bound = attn_error(got[rows], ref[rows], w.dtype)
+    assert err <= bound, f"{w.name} {w.dtype}: error {err:.3e} above {bound:.3e}"
+    assert not torch.isnan(out[:T]).any()
+    # rows past T are left as they were
+    assert torch.isnan(out_full[T:]).all()
+    # fused CLS equals the first row of every sequence, bit for bit
+    assert torch.equal(cls, out[torch.from_numpy(cu[:-1]).long().cuda()])
+    return err
+
+
+@pytest.mark.parametrize("dtype", ["f16", "bf16", "f32"])
+def test_tiny_all_elements(dtype):
+    check_against_oracle(synthetic.tiny(dtype))
+
+
+@pytest.mark.parametrize("dtype", ["f16", "bf16", "f32"])
+def test_tile_edge_lengths(dtype):
+    lengths = [1, 2, 15, 16, 17, 31, 32, 33, 63, 64, 65, 127, 128, 129, 191, 192, 193, 200]
+    w = synthetic.make_workload("edges", len(lengths), 200, 3, lengths, dtype, 77)
+    check_against_oracle(w)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f16"])
+def test_hires_lengths_576_577(dtype):
+    w = synthetic.make_workload("hires_edges", 3, 577, 2, [577, 576, 300], dtype, 78)
+    check_against_oracle(w)
+
+
+def test_deit_b_pruned80_all_sequences():
+    check_against_oracle(synthetic.deit_b_pruned80())
+
+
+@pytest.mark.parametrize("B", synthetic.SERVING_BATCHES)
+@pytest.mark.parametrize("rate", synthetic.SERVING_RATES)
+def test_serving_all_sequences(B, rate):
+    check_against_oracle(synthetic.serving(B, rate))
+
+
+def test_hires_384_sampled():
+    w = synthetic.hires_384()
+    check_against_oracle(w, seqs=sample_sequences(w.lengths, 6))
+
+
+@pytest.mark.parametrize("rate", [0.0, 0.5, 0.9])
+def test_sweep_b512_sampled(rate):
+    w = synthetic.sweep(rate)
+    check_against_oracle(w, seqs=sample_sequences(w.lengths, 8, seed=int(rate * 10)))
+
+
+@pytest.mark.parametrize("dtype", ["f16", "bf16", "f32"])
+def test_separate_qkv_and_padded_output_rows(dtype):
+    w = synthetic.make_workload("layout", 5, 130, 4, [130, 1, 64, 65, 99], dtype, 79)
+    check_against_oracle(w, separate_qkv=True, out_pad=64 if dtype != "f32" else 32)
+
+
+@pytest.mark.parametrize("dtype", ["f16", "bf16", "f32"])
+def test_deterministic(dtype):
+    w = synthetic.make_workload("det", 6, 197, 6, [197, 40, 88, 3, 150, 64], dtype, 80)
+    _, out1, cls1, _ = run_pipeline(w)
+    _, out2, cls2, _ = run_pipeline(w)
+    T = int(w.lengths.sum())
+    assert torch.equal(out1[:T], out2[:T]) and torch.equal(cls1, cls2)
+
+
+def test_bad_cu_seqlens_are_flagged_and_skipped():
+    H, d = 2, 64
+    q = torch.randn(100, H, d, device="cuda", dtype=torch.float16)
+    out = torch.full((100, H, d), 7.0, dtype=torch.float16, device="cuda")
+    rv.ragged_get_device_status()
+    # sequence 0 is longer than the host bound; sequence 1 has a negative length
+    cu = torch.tensor([0, 80, 60], dtype=torch.int32, device="cuda")
+    rv.ragged_attn_fwd(q, q, q, cu, max_seqlen=64, out=out)
+    assert rv.ragged_get_device_status() & rv.RAGGED_DEV_BAD_SEQLENS
+    assert torch.all(out == 7.0)
+    assert rv.ragged_get_device_status() == 0     # reading clears the word
+
+
+def test_pipeline_call_and_graph_replay_match_separate_calls():
+    w = synthetic.serving(4, 0.25)
+    cu_ref, out_ref, cls_ref, _ = run_pipeline(w)
+    p = rv.Pipeline(w.B, w.L_full, w.H, torch.float16)
+    p.dense_qkv.copy_(to_device(w.qkv, "f16"))
+    p.keep.copy_(torch.from_numpy(w.keep))
+    p()
+    torch.cuda.synchronize()
+    T = int(cu_ref[-1])
+    assert np.array_equal(p.cu_seqlens.cpu().numpy(), cu_ref)
+    assert torch.equal(p.out[:T], out_ref[:T]) and torch.equal(p.cls_out, cls_ref)
+    p.cls_out.zero_()
+    p.capture()
+    p.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(p.cls_out, cls_ref)
+    # new inputs written into the same buffers are picked up by the replay
+    w2 = synthetic.serving(4, 0.25, copy=1)
+    p.dense_qkv.copy_(to_device(w2.qkv, "f16"))
+    p.keep.copy_(torch.from_numpy(w2.keep))
+    p.replay()
+    torch.cuda.synchronize()
+    _, out2, cls2, _ = run_pipeline(w2)
+    assert torch.equal(p.cls_out, cls2)
+
+
+def test_ragged_pipeline_binding():
+    w = synthetic.deit_b_pruned80()
+    cu_ref, out_ref, cls_ref, _ = run_pipeline(w)
+    packed, cu, out, cls = rv.ragged_pipeline(to_device(w.qkv, w.dtype), torch.from_numpy(w.keep).cuda())
+    torch.cuda.synchronize()
+    T = int(cu_ref[-1])
+    assert np.array_equal(cu.cpu().numpy(), cu_ref)
+    assert torch.equal(out[:T], out_ref[:T]) and torch.equal(cls, cls_ref)
