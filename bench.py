@@ -132,6 +132,16 @@ def attn_bytes(w) -> int:
     return 4 * w.T * w.H * w.d * e + 4 * (w.B + 1) + w.B * w.H * w.d * e
 
 
+def fused_bytes(w, packed_written: bool = True) -> int:
+    """Algorithmic bytes of one fused pipeline launch: the mask, the kept dense
+    q/k/v rows read once, the packed rows written (when materialised), the
+    attention output and CLS rows written, cu_seqlens written."""
+    e = w.elem_bytes
+    rows = w.T * w.row_bytes
+    return (w.B * w.L_full + rows * (2 if packed_written else 1) + w.T * w.H * w.d * e
+            + w.B * w.H * w.d * e + 4 * (w.B + 1))
+
+
 def pack_bytes(w) -> int:
     """Algorithmic bytes of one pack launch: the mask, the kept rows read and
     written, cu_seqlens written."""
@@ -155,7 +165,7 @@ def run_ours(args, rank, world, dist):
     pipes = {c: [] for c in range(ncopies)}
     for c in range(ncopies):
         for w in workloads[c]:
-            pl = rv.Pipeline(w.B, w.L_full, w.H, torch.float16, device=dev)
+            pl = rv.Pipeline(w.B, w.L_full, w.H, torch.float16, device=dev, flags=rv.RAGGED_PIPELINE_FUSED)
             pl.dense_qkv.copy_(torch.from_numpy(w.qkv).to(dev))
             pl.keep.copy_(torch.from_numpy(w.keep).to(dev))
             pl.bind_inputs(pl.dense_qkv, pl.keep)
@@ -165,7 +175,7 @@ def run_ours(args, rank, world, dist):
     def step(s):
         for pl in pipes[s % ncopies]:
             pl()
-            torch.cuda.synchronize()
+            stream.synchronize()
 
     for s in range(args.warmup):
         step(s)
@@ -211,7 +221,7 @@ def run_ours(args, rank, world, dist):
             pl()
             h1 = time.perf_counter()
             b.record(stream)
-            torch.cuda.synchronize()
+            stream.synchronize()
             t1 = time.perf_counter()
             host.append((h1 - h0) * 1e6)
             dev_t.append(a.elapsed_time(b) * 1e3)
@@ -236,7 +246,7 @@ def run_ours(args, rank, world, dist):
         for s in range(args.steps):
             for pl in pipes[s % ncopies]:
                 pl.replay()
-                torch.cuda.synchronize()
+                stream.synchronize()
         g1.record(stream)
         torch.cuda.synchronize()
         graph_us = g0.elapsed_time(g1) * 1000.0 / (args.steps * len(CASES))
@@ -260,7 +270,7 @@ def run_ours(args, rank, world, dist):
             pl.keep.copy_(keep_h, non_blocking=True)
             pl()
             cls_h.copy_(pl.cls_out, non_blocking=True)
-            torch.cuda.synchronize()
+            stream.synchronize()
 
     for s in range(args.warmup):
         e2e_step(s)
@@ -328,20 +338,32 @@ def run_ours(args, rank, world, dist):
         torch.cuda.synchronize()
         return a.elapsed_time(b) / 1000.0 / (replays * len(launchers))
 
+    def pipeline_launcher(pl):
+        def launch(strm):
+            pl.bind_inputs(pl.dense_qkv, pl.keep, stream=strm)
+            pl()
+            pl.bind_inputs(pl.dense_qkv, pl.keep)
+        return launch
+
     all_pw = [(pipes[c][i], workloads[c][i]) for c in range(ncopies) for i in range(len(CASES))]
+    t_fused = graph_time([pipeline_launcher(p_) for p_, _ in all_pw])
+    b_fused = float(np.mean([fused_bytes(w_) for _, w_ in all_pw]))
     t_attn = graph_time([attn_launcher(p_, w_) for p_, w_ in all_pw])
     t_pack = graph_time([pack_launcher(p_, w_) for p_, w_ in all_pw])
     b_attn = float(np.mean([attn_bytes(w_) for _, w_ in all_pw]))
     b_pack = float(np.mean([pack_bytes(w_) for _, w_ in all_pw]))
     flops = float(np.mean([w_.useful_flops() for _, w_ in all_pw]))
-    roofline = {"bound": "hbm", "achieved": round(b_attn / t_attn / 1e9, 2), "peak": hbm_peak,
-                "unit": "GB/s", "frac": round(b_attn / t_attn / 1e9 / hbm_peak, 4), "traffic": None,
-                "kernel": "attn_fwd_kernel<__half>", "avg_launch_us": round(t_attn * 1e6, 3),
-                "bytes_per_launch": int(b_attn), "launches_timed": 3 * len(all_pw), "peak_kind": peak_kind,
+    roofline = {"bound": "hbm", "achieved": round(b_fused / t_fused / 1e9, 2), "peak": hbm_peak,
+                "unit": "GB/s", "frac": round(b_fused / t_fused / 1e9 / hbm_peak, 4), "traffic": None,
+                "kernel": "attn_resident_kernel<__half, DenseRows> (fused pack + attention + CLS)",
+                "avg_launch_us": round(t_fused * 1e6, 3), "bytes_per_launch": int(b_fused),
+                "launches_timed": 3 * len(all_pw), "peak_kind": peak_kind,
                 "timing": "CUDA graph of back-to-back launches over all input copies, CUDA events",
-                "useful_tflops": round(flops / t_attn / 1e12, 4),
-                "pack_kernel": {"avg_launch_us": round(t_pack * 1e6, 3), "bytes_per_launch": int(b_pack),
-                                "achieved_GBps": round(b_pack / t_pack / 1e9, 2)}}
+                "useful_tflops": round(flops / t_fused / 1e12, 4),
+                "split_path": {"attention_us": round(t_attn * 1e6, 3), "attention_bytes": int(b_attn),
+                               "attention_GBps": round(b_attn / t_attn / 1e9, 2),
+                               "pack_us": round(t_pack * 1e6, 3), "pack_bytes": int(b_pack),
+                               "pack_GBps": round(b_pack / t_pack / 1e9, 2)}}
 
     # ---- larger workloads: attention roofline (single GPU, same kernel family) ----
     larger = {}
@@ -355,7 +377,8 @@ def run_ours(args, rank, world, dist):
             ws = [make(c) for c in range(copies)]
             pls = []
             for w in ws:
-                pl = rv.Pipeline(w.B, w.L_full, w.H, torch.float16 if w.dtype == "f16" else torch.bfloat16, device=dev)
+                pl = rv.Pipeline(w.B, w.L_full, w.H, torch.float16 if w.dtype == "f16" else torch.bfloat16, device=dev,
+                                 flags=rv.RAGGED_PIPELINE_SPLIT)
                 pl.dense_qkv.view(torch.int16).copy_(torch.from_numpy(w.qkv.view(np.int16)).to(dev))
                 pl.keep.copy_(torch.from_numpy(w.keep).to(dev))
                 pl()
@@ -380,7 +403,7 @@ def run_ours(args, rank, world, dist):
     if rank == 0 and world == 1 and not args.quick:
         cpu = cpu_baseline(min_seconds=10.0)
 
-    gpu_launches = 2 * args.steps * len(CASES)
+    gpu_launches = 1 * args.steps * len(CASES)   # one fused launch per call
     hw = {"metric": "ragged attn µs/call (host+device) at BS1-4; useful TFLOP/s & % roofline",
           "value": round(us_per_call, 3), "unit": "µs/call", "n_gpus": world, "steps": args.steps,
           "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 4), "higher_is_better": False,
@@ -388,7 +411,7 @@ def run_ours(args, rank, world, dist):
           "config": {"workload": "serving_deit_s_b1-4_p0-80", "B": list(synthetic.SERVING_BATCHES),
                      "prune_rates": list(synthetic.SERVING_RATES), "jitter": 0.10, "L_full": 197,
                      "heads": 6, "head_dim": 64, "calls_per_step": len(CASES),
-                     "call": "ragged_pipeline (pack + attention with fused CLS) + stream sync",
+                     "call": "ragged_pipeline, fused mode (one launch: pack, attention, CLS) + stream sync",
                      "l2": f"inputs rotated over {ncopies} copies ({ncopies * per_copy / 2**20:.0f} MiB > 2x L2)",
                      "parallelism": "replicas" if world > 1 else "single"},
           "e2e": {"value": round(e2e_us, 3), "unit": "µs/call", "h2d_bytes_per_step": int(h2d),
@@ -433,7 +456,7 @@ def padded_baseline(args, pipes, workloads, ncopies, stream):
             torch.cuda.synchronize()
             t0 = time.perf_counter()
             cls = call(pipes[c][i], Lmax)
-            torch.cuda.synchronize()
+            stream.synchronize()
             if r >= 3:
                 tot.append((time.perf_counter() - t0) * 1e6)
         ref = pipes[0][i].cls_out.float()

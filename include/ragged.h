@@ -120,6 +120,10 @@ RAGGED_API ragged_status ragged_pack(const void *dense, int64_t B, int64_t L_ful
  *   max_seqlen     host-side upper bound on every L_b (e.g. L_full), 1 ..
  *                  RAGGED_MAX_TOKENS.  Sizes the launch; a sequence longer
  *                  than this is skipped and RAGGED_DEV_BAD_SEQLENS is set.
+ *                  Small launches (few sequences x heads) with max_seqlen up
+ *                  to 640, and max_seqlen up to 64, keep each sequence's K
+ *                  and V resident in shared memory (one load burst, keys split
+ *                  across warps); other launches stream K/V tiles.
  *   H, head_dim    heads (>= 1) and head dimension (only 64 is implemented:
  *                  other values return RAGGED_ERR_UNSUPPORTED).
  *   scale          softmax scale, positive and finite; usually 1/sqrt(head_dim).
@@ -165,19 +169,37 @@ RAGGED_API ragged_status ragged_unpack(const void *packed, const int32_t *cu_seq
                             int64_t B, int64_t L_full, int64_t row_bytes, void *dense_out,
                             void *stream);
 
+/* ragged_pipeline modes (flags). */
+#define RAGGED_PIPELINE_AUTO 0u  /* choose per shape (see below)                  */
+#define RAGGED_PIPELINE_FUSED 1u /* one launch: pack, attention and CLS together    */
+#define RAGGED_PIPELINE_SPLIT 2u /* two launches: ragged_pack, then ragged_attn_fwd */
+
 /*
- * ragged_pipeline - pack -> attend -> CLS in one host call (two launches).
+ * ragged_pipeline - pack -> attend -> CLS in one host call.
+ * Paper: radpulse section "Integrated pack pipeline, 2.24x end-to-end"
+ * (cu_seqlens, survivor copy, attention, CLS extraction), and the abstract's
+ * pack-attend-unpack pipeline.
+ *
  * dense_qkv is one fused [B, L_full, 3, H, head_dim] buffer (q, k, v along
- * the third axis); it is packed into packed_qkv [B * L_full, 3, H, head_dim]
- * (capacity), attention reads the packed rows, and writes out [T, H,
- * head_dim] (capacity B * L_full rows) and, if cls_out is not NULL, cls_out
- * [B, H * head_dim].  Requirements as for ragged_pack and ragged_attn_fwd,
- * with max_seqlen = L_full.
+ * the third axis) in `dtype`.  Outputs: cu_seqlens [B + 1]; out [T, H,
+ * head_dim] (capacity B * L_full rows, token stride H * head_dim); cls_out
+ * [B, H * head_dim] unless NULL; packed_qkv [B * L_full (capacity), 3, H,
+ * head_dim] (the survivors' rows, as ragged_pack writes them).
+ *
+ * Fused mode (f16 / bf16, L_full <= 640): a single launch in which every CTA
+ * ranks its image's keep mask, gathers its rows straight from dense_qkv and
+ * writes cu_seqlens, out and cls_out; packed_qkv is optional there (NULL: the
+ * packed q/k/v is not materialised).  Split mode: ragged_pack into packed_qkv
+ * (required) followed by ragged_attn_fwd.  AUTO picks the fused mode when it
+ * is available and B is small enough that every CTA counting the survivors of
+ * the images before its own stays cheap; otherwise the split mode.  Results
+ * are identical in both modes.  Requirements as for ragged_pack and
+ * ragged_attn_fwd, with max_seqlen = L_full and scale positive and finite.
  */
 RAGGED_API ragged_status ragged_pipeline(const void *dense_qkv, const uint8_t *keep, int64_t B,
-                              int64_t L_full, int64_t H, int64_t head_dim, float scale,
-                              ragged_dtype dtype, void *packed_qkv, int32_t *cu_seqlens,
-                              void *out, void *cls_out, void *stream);
+                                         int64_t L_full, int64_t H, int64_t head_dim, float scale,
+                                         ragged_dtype dtype, void *packed_qkv, int32_t *cu_seqlens,
+                                         void *out, void *cls_out, uint32_t flags, void *stream);
 
 /*
  * ragged_get_device_status - read and clear the status word of the current

@@ -34,6 +34,9 @@ RAGGED_ERR_DEVICE = 4
 RAGGED_DEV_BAD_SEQLENS = 0x1
 RAGGED_DEV_TIMEOUT = 0x2
 RAGGED_MAX_TOKENS = 16384
+RAGGED_PIPELINE_AUTO = 0
+RAGGED_PIPELINE_FUSED = 1
+RAGGED_PIPELINE_SPLIT = 2
 
 DTYPE_CODES = {torch.float16: 0, torch.bfloat16: 1, torch.float32: 2}
 DTYPE_NAMES = {"f16": torch.float16, "bf16": torch.bfloat16, "f32": torch.float32}
@@ -66,7 +69,7 @@ def load(path: Optional[str] = None):
     lib.ragged_attn_fwd.argtypes = [vp, vp, vp, i64, i64, vp, i64, i64, i64, i64, f32, i32, vp, i64, vp, vp]
     lib.ragged_unpack_cls.argtypes = [vp, vp, i64, i64, vp, vp]
     lib.ragged_unpack.argtypes = [vp, vp, vp, i64, i64, i64, vp, vp]
-    lib.ragged_pipeline.argtypes = [vp, vp, i64, i64, i64, i64, f32, i32, vp, vp, vp, vp, vp]
+    lib.ragged_pipeline.argtypes = [vp, vp, i64, i64, i64, i64, f32, i32, vp, vp, vp, vp, ctypes.c_uint32, vp]
     lib.ragged_get_device_status.argtypes = [ctypes.POINTER(ctypes.c_uint32), vp]
     for name in ("ragged_pack", "ragged_attn_fwd", "ragged_unpack_cls", "ragged_unpack",
                  "ragged_pipeline", "ragged_get_device_status"):
@@ -189,11 +192,15 @@ def ragged_unpack(packed: torch.Tensor, cu_seqlens: torch.Tensor, keep: torch.Te
 
 
 def ragged_pipeline(dense_qkv: torch.Tensor, keep: torch.Tensor, scale: Optional[float] = None,
-                    packed_qkv=None, cu_seqlens=None, out=None, cls_out=None, stream=None):
-    """dense_qkv [B, L_full, 3, H, 64] -> (packed_qkv, cu_seqlens, out [cap, H, 64], cls_out [B, H, 64])."""
+                    packed_qkv=None, cu_seqlens=None, out=None, cls_out=None,
+                    flags: int = RAGGED_PIPELINE_AUTO, materialize_packed: bool = True, stream=None):
+    """dense_qkv [B, L_full, 3, H, 64] -> (packed_qkv or None, cu_seqlens, out [cap, H, 64], cls_out [B, H, 64]).
+
+    With materialize_packed=False the fused mode does not write the packed q/k/v.
+    """
     B, L_full, three, H, d = dense_qkv.shape
     dev, dt = dense_qkv.device, dense_qkv.dtype
-    if packed_qkv is None:
+    if packed_qkv is None and materialize_packed:
         packed_qkv = torch.empty((B * L_full, 3, H, d), dtype=dt, device=dev)
     if cu_seqlens is None:
         cu_seqlens = torch.empty(B + 1, dtype=torch.int32, device=dev)
@@ -205,7 +212,7 @@ def ragged_pipeline(dense_qkv: torch.Tensor, keep: torch.Tensor, scale: Optional
         scale = d ** -0.5
     _check(load().ragged_pipeline(_ptr(dense_qkv), _ptr(keep), B, L_full, H, d, float(scale),
                                   _dtype_code(dense_qkv), _ptr(packed_qkv), _ptr(cu_seqlens), _ptr(out),
-                                  _ptr(cls_out), _stream(stream)))
+                                  _ptr(cls_out), int(flags), _stream(stream)))
     return packed_qkv, cu_seqlens, out, cls_out
 
 
@@ -225,13 +232,16 @@ class Pipeline:
     """
 
     def __init__(self, B: int, L_full: int, H: int, dtype: torch.dtype, device="cuda",
-                 scale: Optional[float] = None, head_dim: int = 64):
+                 scale: Optional[float] = None, head_dim: int = 64, flags: int = RAGGED_PIPELINE_AUTO,
+                 materialize_packed: bool = True):
         self.B, self.L_full, self.H, self.d = B, L_full, H, head_dim
         self.dtype = dtype
+        self.flags = flags
         dev = torch.device(device)
         self.dense_qkv = torch.empty((B, L_full, 3, H, head_dim), dtype=dtype, device=dev)
         self.keep = torch.empty((B, L_full), dtype=torch.uint8, device=dev)
-        self.packed_qkv = torch.empty((B * L_full, 3, H, head_dim), dtype=dtype, device=dev)
+        self.packed_qkv = (torch.empty((B * L_full, 3, H, head_dim), dtype=dtype, device=dev)
+                           if materialize_packed else None)
         self.cu_seqlens = torch.empty(B + 1, dtype=torch.int32, device=dev)
         self.out = torch.empty((B * L_full, H, head_dim), dtype=dtype, device=dev)
         self.cls_out = torch.empty((B, H, head_dim), dtype=dtype, device=dev)
@@ -246,9 +256,9 @@ class Pipeline:
         c = ctypes
         self._args = (c.c_void_p(dense_qkv.data_ptr()), c.c_void_p(keep.data_ptr()), c.c_int64(self.B),
                       c.c_int64(self.L_full), c.c_int64(self.H), c.c_int64(self.d), c.c_float(self.scale),
-                      c.c_int(DTYPE_CODES[self.dtype]), c.c_void_p(self.packed_qkv.data_ptr()),
+                      c.c_int(DTYPE_CODES[self.dtype]), c.c_void_p(_ptr(self.packed_qkv)),
                       c.c_void_p(self.cu_seqlens.data_ptr()), c.c_void_p(self.out.data_ptr()),
-                      c.c_void_p(self.cls_out.data_ptr()), c.c_void_p(_stream(stream)))
+                      c.c_void_p(self.cls_out.data_ptr()), c.c_uint32(self.flags), c.c_void_p(_stream(stream)))
         self._fn = load().ragged_pipeline
 
     def __call__(self) -> None:

@@ -23,7 +23,7 @@
 // bf16's 2^-9; this keeps the result within the rounding of the bf16 output.
 #pragma once
 
-#include "common.cuh"
+#include "mma_common.cuh"
 
 namespace ragged {
 namespace mma_attn {
@@ -35,70 +35,6 @@ constexpr int kWarps = 4;
 constexpr int kThreads = kWarps * 32;
 constexpr int kTileBytes = kBlockM * kHeadDim * 2;   // 8 KB per 64 x 64 16-bit tile
 constexpr int kSmemBytes = kTileBytes * 5;            // Q, K[2], V[2]
-
-// Byte offset of 16-byte chunk `c` (0..7) of row `r` in a [64][64] 16-bit tile;
-// chunks are XOR-swizzled by row so ldmatrix on 8 rows hits 8 distinct banks.
-__device__ __forceinline__ uint32_t swz(int r, int c) {
-    return static_cast<uint32_t>(r * 128 + ((c ^ (r & 7)) << 4));
-}
-
-__device__ __forceinline__ void ldmatrix_x4(uint32_t (&d)[4], uint32_t addr) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
-                 : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
-                 : "r"(addr));
-}
-__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t (&d)[4], uint32_t addr) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
-                 : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
-                 : "r"(addr));
-}
-
-template <typename T>
-struct Mma;
-
-template <>
-struct Mma<__half> {
-    __device__ __forceinline__ static void run(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
-                                               uint32_t b1) {
-        asm volatile(
-            "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-            "{%8,%9}, {%0,%1,%2,%3};\n"
-            : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-            : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-    }
-    __device__ __forceinline__ static uint32_t pack(float lo, float hi) {
-        __half2 h = __floats2half2_rn(lo, hi);
-        return *reinterpret_cast<uint32_t*>(&h);
-    }
-};
-
-template <>
-struct Mma<__nv_bfloat16> {
-    __device__ __forceinline__ static void run(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
-                                               uint32_t b1) {
-        asm volatile(
-            "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-            "{%8,%9}, {%0,%1,%2,%3};\n"
-            : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-            : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-    }
-    __device__ __forceinline__ static uint32_t pack(float lo, float hi) {
-        __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
-        return *reinterpret_cast<uint32_t*>(&h);
-    }
-    // Residual of the bf16 rounding of (lo, hi), rounded to bf16 again.
-    __device__ __forceinline__ static uint32_t pack_residual(float lo, float hi, uint32_t rounded) {
-        __nv_bfloat162 r = *reinterpret_cast<__nv_bfloat162*>(&rounded);
-        const float2 f = __bfloat1622float2(r);
-        return pack(lo - f.x, hi - f.y);
-    }
-};
-
-__device__ __forceinline__ float fast_exp2(float x) {
-    float y;
-    asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
-    return y;
-}
 
 // Loads rows [row0, row0 + 64) of one head of one sequence into a swizzled
 // shared tile.  `g` points at element (row 0, head h, dim 0).

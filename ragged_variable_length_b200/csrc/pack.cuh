@@ -28,38 +28,41 @@ constexpr int kPackUnroll = 4;
 __device__ __forceinline__ int nonzero_bytes(uint32_t w) { return __popc(__vcmpne4(w, 0u)) >> 3; }
 
 // Nonzero bytes in p[0, n) plus every thread's `extra`, summed over the CTA
-// (result in every thread).
+// of NT threads (result in every thread).  s_red holds NT / 32 ints.
+template <int NT>
 __device__ __forceinline__ int cta_count_nonzero(const uint8_t* __restrict__ p, int64_t n,
                                                  int extra, int* s_red) {
     const int tid = threadIdx.x;
     int cnt = extra;
     int64_t head = (16 - (reinterpret_cast<uintptr_t>(p) & 15)) & 15;
     if (head > n) head = n;
-    for (int64_t i = tid; i < head; i += kPackThreads) cnt += p[i] != 0;
+    for (int64_t i = tid; i < head; i += NT) cnt += p[i] != 0;
     const uint4* v = reinterpret_cast<const uint4*>(p + head);
     const int64_t nv = (n - head) >> 4;
-    for (int64_t i = tid; i < nv; i += kPackThreads) {
+    for (int64_t i = tid; i < nv; i += NT) {
         const uint4 x = __ldg(v + i);
         cnt += nonzero_bytes(x.x) + nonzero_bytes(x.y) + nonzero_bytes(x.z) + nonzero_bytes(x.w);
     }
-    for (int64_t i = head + nv * 16 + tid; i < n; i += kPackThreads) cnt += p[i] != 0;
+    for (int64_t i = head + nv * 16 + tid; i < n; i += NT) cnt += p[i] != 0;
     cnt = warp_sum(cnt);
     if ((tid & 31) == 0) s_red[tid >> 5] = cnt;
     __syncthreads();
     int total = 0;
 #pragma unroll
-    for (int w = 0; w < kPackThreads / 32; ++w) total += s_red[w];
+    for (int w = 0; w < NT / 32; ++w) total += s_red[w];
     __syncthreads();
     return total;
 }
 
-// Ranks the survivors of one image: s_kept[r] = token index of the r-th
-// survivor (CLS at r = 0).  Returns the survivor count L_b.
+// Ranks the survivors of one image with a CTA of NT threads: s_kept[r] =
+// token index of the r-th survivor (CLS at r = 0).  Returns the survivor
+// count L_b (in every thread).
+template <int NT>
 __device__ __forceinline__ int cta_rank_survivors(const uint8_t* __restrict__ kb, int L_full,
                                                   int* s_kept, int* s_red) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     int running = 0;
-    for (int j0 = 0; j0 < L_full; j0 += kPackThreads) {
+    for (int j0 = 0; j0 < L_full; j0 += NT) {
         const int j = j0 + tid;
         const bool kept = j < L_full && (j == 0 || kb[j] != 0);
         const unsigned bal = __ballot_sync(0xffffffffu, kept);
@@ -67,7 +70,7 @@ __device__ __forceinline__ int cta_rank_survivors(const uint8_t* __restrict__ kb
         __syncthreads();
         int before = 0, total = 0;
 #pragma unroll
-        for (int w = 0; w < kPackThreads / 32; ++w) {
+        for (int w = 0; w < NT / 32; ++w) {
             const int x = s_red[w];
             before += (w < warp) ? x : 0;
             total += x;
@@ -127,9 +130,9 @@ __global__ void __launch_bounds__(kPackThreads)
     int forced = 0;
     for (int i = threadIdx.x; i < b; i += kPackThreads)
         forced += keep[static_cast<int64_t>(i) * L_full] == 0;
-    const int base = cta_count_nonzero(keep, prev, forced, s_red);
+    const int base = cta_count_nonzero<kPackThreads>(keep, prev, forced, s_red);
 
-    const int L_b = cta_rank_survivors(keep + prev, L_full, s_kept, s_red);
+    const int L_b = cta_rank_survivors<kPackThreads>(keep + prev, L_full, s_kept, s_red);
     if (split == 0 && threadIdx.x == 0) {
         cu[b + 1] = base + L_b;
         if (b == 0) cu[0] = 0;
@@ -151,7 +154,7 @@ __global__ void __launch_bounds__(kPackThreads)
     const int b = blockIdx.y;
     const int split = blockIdx.x, splits = gridDim.x;
     const int64_t prev = static_cast<int64_t>(b) * L_full;
-    const int L_b = cta_rank_survivors(keep + prev, L_full, s_kept, s_red);
+    const int L_b = cta_rank_survivors<kPackThreads>(keep + prev, L_full, s_kept, s_red);
     const int base = __ldg(cu + b);
     if (base < 0 || __ldg(cu + b + 1) - base != L_b) {
         if (threadIdx.x == 0) raise_status(RAGGED_DEV_BAD_SEQLENS);

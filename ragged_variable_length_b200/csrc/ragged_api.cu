@@ -11,6 +11,7 @@
 
 #include "attn_f32.cuh"
 #include "attn_mma.cuh"
+#include "attn_resident.cuh"
 #include "common.cuh"
 #include "pack.cuh"
 
@@ -98,6 +99,59 @@ int pack_splits(int64_t B, int64_t L_full) {
 
 bool g_pack_smem[kMaxDevices], g_unpack_smem[kMaxDevices];
 bool g_mma_f16_smem[kMaxDevices], g_mma_bf16_smem[kMaxDevices], g_f32_smem[kMaxDevices];
+
+// Largest dynamic shared memory of the resident kernels: 640 keys and a
+// 640-entry survivor list.
+constexpr int kResidentSmemMax = ragged::resident::smem_bytes(ragged::resident::kMaxKeyTiles,
+                                                              ragged::resident::kMaxKeys);
+
+// Warps per row block in the resident kernel: split the keys of a sequence
+// across warps when the launch is too small to fill the GPU twice over with
+// 64-row tiles (the latency-bound serving regime); keep 64-row tiles otherwise.
+int resident_ksplit(int64_t B, int64_t H, int key_tiles) {
+    if (key_tiles <= 1) return 1;
+    const int64_t ctas64 = static_cast<int64_t>(key_tiles) * H * B;
+    if (ctas64 >= 2LL * sm_count()) return 1;
+    return key_tiles == 2 ? 2 : 4;
+}
+
+template <typename T, class Src, int KS>
+ragged_status launch_resident_ks(const Src& src, int64_t B, int64_t H, int key_tiles, int list_entries,
+                                 float scale, void* out, int64_t out_tok_stride, void* cls_out, void* packed_out,
+                                 bool (&smem_done)[kMaxDevices], cudaStream_t s) {
+    using namespace ragged::resident;
+    auto kernel = attn_resident_kernel<T, Src, KS>;
+    ragged_status st = ensure_smem(kernel, kResidentSmemMax, smem_done);
+    if (st != RAGGED_OK) return st;
+    constexpr int rows = 16 * (kWarps / KS);
+    const int64_t max_rows = static_cast<int64_t>(key_tiles) * kBlockN;
+    const dim3 grid(static_cast<unsigned>((max_rows + rows - 1) / rows), static_cast<unsigned>(H),
+                    static_cast<unsigned>(B));
+    kernel<<<grid, kThreads, smem_bytes(key_tiles, list_entries), s>>>(
+        src, key_tiles, scale * 1.4426950408889634f, static_cast<int>(H), static_cast<uint16_t*>(out),
+        out_tok_stride, static_cast<uint16_t*>(cls_out), static_cast<uint16_t*>(packed_out));
+    return cuda_check(cudaGetLastError(), "resident attention launch");
+}
+
+// slot: 0/1 packed f16/bf16, 2/3 dense f16/bf16 (one set of smem flags per kernel).
+bool g_res_smem_ks[4][3][kMaxDevices];
+
+template <typename T, class Src>
+ragged_status launch_resident(const Src& src, int64_t B, int64_t H, int key_tiles, int list_entries,
+                              float scale, void* out, int64_t out_tok_stride, void* cls_out, void* packed_out,
+                              int slot, cudaStream_t s) {
+    switch (resident_ksplit(B, H, key_tiles)) {
+        case 4:
+            return launch_resident_ks<T, Src, 4>(src, B, H, key_tiles, list_entries, scale, out, out_tok_stride,
+                                                 cls_out, packed_out, g_res_smem_ks[slot][2], s);
+        case 2:
+            return launch_resident_ks<T, Src, 2>(src, B, H, key_tiles, list_entries, scale, out, out_tok_stride,
+                                                 cls_out, packed_out, g_res_smem_ks[slot][1], s);
+        default:
+            return launch_resident_ks<T, Src, 1>(src, B, H, key_tiles, list_entries, scale, out, out_tok_stride,
+                                                 cls_out, packed_out, g_res_smem_ks[slot][0], s);
+    }
+}
 
 }  // namespace
 
@@ -224,6 +278,21 @@ ragged_status ragged_attn_fwd(const void* q, const void* k, const void* v, int64
             static_cast<float*>(out), out_tok_stride, static_cast<float*>(cls_out));
         return cuda_check(cudaGetLastError(), "attention (f32) launch");
     }
+    // Whole-sequence residency pays off in the latency-bound regime (few CTAs:
+    // keys split across warps) and for single-tile sequences; large launches
+    // of longer sequences keep more CTAs per SM with the streaming kernel.
+    const int res_tiles = static_cast<int>((max_seqlen + 63) / 64);
+    if (max_seqlen <= ragged::resident::kMaxKeys &&
+        (res_tiles == 1 || resident_ksplit(B, H, res_tiles) > 1)) {
+        ragged::resident::PackedRows src{static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(k),
+                                         static_cast<const uint16_t*>(v), tok_stride, head_stride, cu_seqlens,
+                                         static_cast<int>(max_seqlen), 0, 0, 0};
+        const int key_tiles = static_cast<int>((max_seqlen + 63) / 64);
+        if (dtype == RAGGED_F16)
+            return launch_resident<__half>(src, B, H, key_tiles, 0, scale, out, out_tok_stride, cls_out, nullptr, 0, s);
+        return launch_resident<__nv_bfloat16>(src, B, H, key_tiles, 0, scale, out, out_tok_stride, cls_out, nullptr,
+                                              1, s);
+    }
     using namespace ragged::mma_attn;
     const dim3 grid(static_cast<unsigned>((max_seqlen + kBlockM - 1) / kBlockM), static_cast<unsigned>(H),
                     static_cast<unsigned>(B));
@@ -249,19 +318,59 @@ ragged_status ragged_attn_fwd(const void* q, const void* k, const void* v, int64
 ragged_status ragged_pipeline(const void* dense_qkv, const uint8_t* keep, int64_t B, int64_t L_full,
                               int64_t H, int64_t head_dim, float scale, ragged_dtype dtype,
                               void* packed_qkv, int32_t* cu_seqlens, void* out, void* cls_out,
-                              void* stream) {
+                              uint32_t flags, void* stream) {
     if (head_dim != 64) return fail(RAGGED_ERR_UNSUPPORTED, "head_dim = %lld (only 64 is implemented)", (long long)head_dim);
     if (H < 1 || H > 65535) return fail(RAGGED_ERR_INVALID_ARG, "H = %lld outside [1, 65535]", (long long)H);
     if (dtype != RAGGED_F16 && dtype != RAGGED_BF16 && dtype != RAGGED_F32)
         return fail(RAGGED_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
+    if ((flags & ~(RAGGED_PIPELINE_FUSED | RAGGED_PIPELINE_SPLIT)) != 0 ||
+        flags == (RAGGED_PIPELINE_FUSED | RAGGED_PIPELINE_SPLIT))
+        return fail(RAGGED_ERR_INVALID_ARG, "flags = %u is not a valid pipeline mode", flags);
     const int64_t esz = dtype == RAGGED_F32 ? 4 : 2;
     const int64_t D = H * head_dim;
-    ragged_status st = ragged_pack(dense_qkv, B, L_full, 3 * D * esz, keep, packed_qkv, cu_seqlens,
-                                   nullptr, stream);
-    if (st != RAGGED_OK || B == 0) return st;
-    const char* base = static_cast<const char*>(packed_qkv);
-    return ragged_attn_fwd(base, base + D * esz, base + 2 * D * esz, 3 * D, head_dim, cu_seqlens, B,
-                           L_full, H, head_dim, scale, dtype, out, D, cls_out, stream);
+    ragged_status st = check_rows(B, L_full, 3 * D * esz);
+    if (st != RAGGED_OK) return st;
+    if (!(scale > 0.f) || scale > 3.0e38f)
+        return fail(RAGGED_ERR_INVALID_ARG, "scale must be a positive finite number");
+    // One fused launch when the whole sequence fits the resident kernel and
+    // the per-CTA survivor counting stays small; pack + attention otherwise.
+    const int64_t key_tiles = (L_full + 63) / 64;
+    const bool fusable = dtype != RAGGED_F32 && L_full <= ragged::resident::kMaxKeys;
+    // Every CTA of image b reads the b * L_full mask bytes before it.
+    const int64_t rows_per_cta = 16 * (4 / resident_ksplit(B, H, static_cast<int>(key_tiles)));
+    const int64_t ctas_per_image = (key_tiles * 64 + rows_per_cta - 1) / rows_per_cta * H;
+    const int64_t count_bytes = ctas_per_image * L_full * (B * B / 2);
+    bool fused = fusable && count_bytes <= (int64_t(32) << 20);
+    if (flags & RAGGED_PIPELINE_FUSED) {
+        if (!fusable) return fail(RAGGED_ERR_UNSUPPORTED, "the fused pipeline needs f16/bf16 and L_full <= %d",
+                                  ragged::resident::kMaxKeys);
+        fused = true;
+    }
+    if (flags & RAGGED_PIPELINE_SPLIT) fused = false;
+    if (!fused) {
+        if (packed_qkv == nullptr)
+            return fail(RAGGED_ERR_INVALID_ARG, "packed_qkv is required when the pipeline runs as two launches");
+        st = ragged_pack(dense_qkv, B, L_full, 3 * D * esz, keep, packed_qkv, cu_seqlens, nullptr, stream);
+        if (st != RAGGED_OK || B == 0) return st;
+        const char* base = static_cast<const char*>(packed_qkv);
+        return ragged_attn_fwd(base, base + D * esz, base + 2 * D * esz, 3 * D, head_dim, cu_seqlens, B,
+                               L_full, H, head_dim, scale, dtype, out, D, cls_out, stream);
+    }
+    if (cu_seqlens == nullptr || (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u))
+        return fail(RAGGED_ERR_INVALID_ARG, "cu_seqlens must be a 4-byte aligned device pointer");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (B == 0) return cuda_check(cudaMemsetAsync(cu_seqlens, 0, sizeof(int32_t), s), "cudaMemsetAsync");
+    if (dense_qkv == nullptr || keep == nullptr || out == nullptr)
+        return fail(RAGGED_ERR_INVALID_ARG, "dense_qkv, keep and out must not be NULL");
+    if (!aligned16(dense_qkv) || !aligned16(out) || !aligned16(cls_out) || !aligned16(packed_qkv))
+        return fail(RAGGED_ERR_INVALID_ARG, "dense_qkv, packed_qkv, out and cls_out must be 16-byte aligned");
+    ragged::resident::DenseRows src{static_cast<const uint16_t*>(dense_qkv), keep, cu_seqlens,
+                                    static_cast<int>(L_full), static_cast<int>(H), 0, 0, 0, 0, nullptr};
+    if (dtype == RAGGED_F16)
+        return launch_resident<__half>(src, B, H, static_cast<int>(key_tiles), static_cast<int>(L_full), scale, out,
+                                       D, cls_out, packed_qkv, 2, s);
+    return launch_resident<__nv_bfloat16>(src, B, H, static_cast<int>(key_tiles), static_cast<int>(L_full), scale,
+                                          out, D, cls_out, packed_qkv, 3, s);
 }
 
 ragged_status ragged_get_device_status(uint32_t* host_out, void* stream) {

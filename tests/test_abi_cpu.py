@@ -129,13 +129,33 @@ def test_unpack_rejects(lib):
     assert lib.ragged_unpack_cls(A16, A16, 0, 48, None, None) == rv.RAGGED_OK
 
 
-def test_pipeline_rejects(lib):
-    assert lib.ragged_pipeline(A16, A16, 2, 197, 6, 32, 0.125, 0, A16, A16, A16, None, None) \
-        == rv.RAGGED_ERR_UNSUPPORTED
-    assert lib.ragged_pipeline(A16, A16, 2, 197, 0, 64, 0.125, 0, A16, A16, A16, None, None) \
-        == rv.RAGGED_ERR_INVALID_ARG
-    assert lib.ragged_pipeline(A8, A16, 2, 197, 6, 64, 0.125, 0, A16, A16, A16, None, None) \
-        == rv.RAGGED_ERR_INVALID_ARG
+def _pipe(lib, **kw):
+    a = dict(dense=A16, keep=A16, B=2, L=197, H=6, d=64, scale=0.125, dt=0, packed=A16, cu=A16, out=A16,
+             cls=None, flags=0)
+    a.update(kw)
+    return lib.ragged_pipeline(a["dense"], a["keep"], a["B"], a["L"], a["H"], a["d"], a["scale"], a["dt"],
+                               a["packed"], a["cu"], a["out"], a["cls"], a["flags"], None)
+
+
+@pytest.mark.parametrize("kw,status,needle", [
+    (dict(d=32), rv.RAGGED_ERR_UNSUPPORTED, "head_dim"),
+    (dict(H=0), rv.RAGGED_ERR_INVALID_ARG, "H ="),
+    (dict(dense=A8), rv.RAGGED_ERR_INVALID_ARG, "16-byte"),
+    (dict(out=A8), rv.RAGGED_ERR_INVALID_ARG, "16-byte"),
+    (dict(flags=3), rv.RAGGED_ERR_INVALID_ARG, "flags"),
+    (dict(flags=8), rv.RAGGED_ERR_INVALID_ARG, "flags"),
+    (dict(scale=0.0), rv.RAGGED_ERR_INVALID_ARG, "scale"),
+    (dict(L=0), rv.RAGGED_ERR_INVALID_ARG, "L_full"),
+    (dict(B=-1), rv.RAGGED_ERR_INVALID_ARG, "negative"),
+    (dict(flags=1, L=641), rv.RAGGED_ERR_UNSUPPORTED, "fused"),
+    (dict(flags=1, dt=2), rv.RAGGED_ERR_UNSUPPORTED, "fused"),
+    (dict(flags=2, packed=None), rv.RAGGED_ERR_INVALID_ARG, "packed_qkv"),
+    (dict(flags=1, cu=None), rv.RAGGED_ERR_INVALID_ARG, "cu_seqlens"),
+    (dict(flags=1, keep=None), rv.RAGGED_ERR_INVALID_ARG, "NULL"),
+])
+def test_pipeline_rejects(lib, kw, status, needle):
+    assert _pipe(lib, **kw) == status
+    assert needle in rv.ragged_last_error()
 
 
 def test_device_status_needs_an_output_pointer(lib):

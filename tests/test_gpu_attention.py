@@ -18,8 +18,11 @@ from helpers import TORCH_DTYPE, attn_error, to_device, to_f64
 pytestmark = pytest.mark.gpu
 
 
-def run_pipeline(w, separate_qkv=False, out_pad=0):
-    """Device pack -> attend (with fused CLS) for a synthetic workload."""
+def run_pipeline(w, separate_qkv=False, out_pad=0, max_seqlen=None):
+    """Device pack -> attend (with fused CLS) for a synthetic workload.
+
+    max_seqlen above 640 selects the streaming attention kernel; the default
+    (L_full) selects the resident one when L_full <= 640."""
     dense = to_device(w.qkv, w.dtype)
     keep = torch.from_numpy(w.keep).cuda()
     packed, cu = rv.ragged_pack(dense, keep)
@@ -32,7 +35,7 @@ def run_pipeline(w, separate_qkv=False, out_pad=0):
         q, k, v = (packed[:, i].contiguous() for i in range(3))
     else:
         q, k, v = packed[:, 0], packed[:, 1], packed[:, 2]
-    rv.ragged_attn_fwd(q, k, v, cu, w.L_full, w.scale, out=out, cls_out=cls)
+    rv.ragged_attn_fwd(q, k, v, cu, max_seqlen or w.L_full, w.scale, out=out, cls_out=cls)
     torch.cuda.synchronize()
     assert rv.ragged_get_device_status() == 0
     return cu.cpu().numpy(), out, cls, out_full
@@ -71,15 +74,31 @@ def test_tiny_all_elements(dtype):
 
 
 @pytest.mark.parametrize("dtype", ["f16", "bf16", "f32"])
-def test_tile_edge_lengths(dtype):
+@pytest.mark.parametrize("kernel", ["resident", "streaming"])
+def test_tile_edge_lengths(dtype, kernel):
     lengths = [1, 2, 15, 16, 17, 31, 32, 33, 63, 64, 65, 127, 128, 129, 191, 192, 193, 200]
     w = synthetic.make_workload("edges", len(lengths), 200, 3, lengths, dtype, 77)
+    check_against_oracle(w, max_seqlen=None if kernel == "resident" else 1000)
+
+
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+def test_long_sequences_streaming_kernel(dtype):
+    """L_full above the resident limit (640 keys) runs the streaming kernel."""
+    w = synthetic.make_workload("long", 4, 1000, 2, [1000, 700, 641, 65], dtype, 81)
     check_against_oracle(w)
 
 
+def test_resident_and_streaming_agree_with_the_bound_unused():
+    """A larger max_seqlen than needed changes the kernel, not the result's accuracy."""
+    w = synthetic.deit_b_pruned80()
+    a = check_against_oracle(w)
+    b = check_against_oracle(w, max_seqlen=2000)
+    assert a < 4e-3 and b < 4e-3
+
+
 @pytest.mark.parametrize("dtype", ["bf16", "f16"])
-def test_hires_lengths_576_577(dtype):
-    w = synthetic.make_workload("hires_edges", 3, 577, 2, [577, 576, 300], dtype, 78)
+def test_hires_lengths_576_577_640(dtype):
+    w = synthetic.make_workload("hires_edges", 4, 640, 2, [577, 576, 300, 640], dtype, 78)
     check_against_oracle(w)
 
 
@@ -93,9 +112,10 @@ def test_serving_all_sequences(B, rate):
     check_against_oracle(synthetic.serving(B, rate))
 
 
-def test_hires_384_sampled():
+@pytest.mark.parametrize("kernel", ["resident", "streaming"])
+def test_hires_384_sampled(kernel):
     w = synthetic.hires_384()
-    check_against_oracle(w, seqs=sample_sequences(w.lengths, 6))
+    check_against_oracle(w, seqs=sample_sequences(w.lengths, 6), max_seqlen=None if kernel == "resident" else 1024)
 
 
 @pytest.mark.parametrize("rate", [0.0, 0.5, 0.9])
