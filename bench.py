@@ -384,13 +384,23 @@ def run_ours(args, rank, world, dist):
                 pl()
                 pls.append(pl)
             torch.cuda.synchronize()
-            t = graph_time([attn_launcher(p_, w_) for p_, w_ in zip(pls, ws)], replays=max(3, 30 // copies))
             bts = float(np.mean([attn_bytes(w_) for w_ in ws]))
             fl = float(np.mean([w_.useful_flops() for w_ in ws]))
             t_roof = max(bts / (hbm_peak * 1e9), fl / (bf16_peak * 1e12))
-            larger[name] = {"avg_launch_us": round(t * 1e6, 2), "GBps": round(bts / t / 1e9, 1),
-                            "useful_tflops": round(fl / t / 1e12, 2), "roofline_frac": round(t_roof / t, 4),
-                            "t_roof_us": round(t_roof * 1e6, 2),
+            per_kernel = {}
+            for kname, kcode in (("streaming", rv.RAGGED_ATTN_STREAMING), ("resident", rv.RAGGED_ATTN_RESIDENT),
+                                 ("tcgen05", rv.RAGGED_ATTN_TCGEN05)):
+                prev = rv.ragged_set_attn_kernel(kcode)
+                try:
+                    t = graph_time([attn_launcher(p_, w_) for p_, w_ in zip(pls, ws)], replays=max(3, 30 // copies))
+                finally:
+                    rv.ragged_set_attn_kernel(prev)
+                per_kernel[kname] = {"avg_launch_us": round(t * 1e6, 2), "GBps": round(bts / t / 1e9, 1),
+                                     "useful_tflops": round(fl / t / 1e12, 2), "roofline_frac": round(t_roof / t, 4)}
+            t = graph_time([attn_launcher(p_, w_) for p_, w_ in zip(pls, ws)], replays=max(3, 30 // copies))
+            larger[name] = {"auto": {"avg_launch_us": round(t * 1e6, 2), "roofline_frac": round(t_roof / t, 4)},
+                            "kernels": per_kernel, "t_roof_us": round(t_roof * 1e6, 2),
+                            "bytes_per_launch": int(bts), "useful_flops": int(fl),
                             "l2": f"inputs rotated over {copies} copies" if copies > 1 else "packed q/k/v exceed L2"}
             del pls
             torch.cuda.empty_cache()

@@ -141,6 +141,24 @@ RAGGED_API ragged_status ragged_attn_fwd(const void *q, const void *k, const voi
                               ragged_dtype dtype, void *out, int64_t out_tok_stride,
                               void *cls_out, void *stream);
 
+/* Attention kernels (ragged_set_attn_kernel). */
+#define RAGGED_ATTN_AUTO 0      /* per launch shape (default)                               */
+#define RAGGED_ATTN_STREAMING 1 /* mma.sync, K/V tiles streamed, any max_seqlen             */
+#define RAGGED_ATTN_RESIDENT 2  /* mma.sync, whole sequence in shared memory, <= 640 keys  */
+#define RAGGED_ATTN_TCGEN05 3   /* tcgen05.mma with TMEM accumulators, K/V streamed        */
+
+/*
+ * ragged_set_attn_kernel - process-wide choice of the f16/bf16 attention
+ * kernel used by ragged_attn_fwd (and by the split mode of ragged_pipeline).
+ * All kernels compute the same operation to the same tolerance; the choice
+ * only changes speed.  Returns the previous choice, or -1 (and changes
+ * nothing) for an unknown value.  A launch whose max_seqlen exceeds what the
+ * chosen kernel holds (640 keys for RAGGED_ATTN_RESIDENT) returns
+ * RAGGED_ERR_UNSUPPORTED.  The fp32 check path
+ * has a single kernel.
+ */
+RAGGED_API int32_t ragged_set_attn_kernel(int32_t kernel);
+
 /*
  * ragged_unpack_cls - CLS extraction (step 3).
  * Paper: radpulse section "Integrated pack pipeline" (after attention and the

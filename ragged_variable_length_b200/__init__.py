@@ -37,13 +37,17 @@ RAGGED_MAX_TOKENS = 16384
 RAGGED_PIPELINE_AUTO = 0
 RAGGED_PIPELINE_FUSED = 1
 RAGGED_PIPELINE_SPLIT = 2
+RAGGED_ATTN_AUTO = 0
+RAGGED_ATTN_STREAMING = 1
+RAGGED_ATTN_RESIDENT = 2
+RAGGED_ATTN_TCGEN05 = 3
 
 DTYPE_CODES = {torch.float16: 0, torch.bfloat16: 1, torch.float32: 2}
 DTYPE_NAMES = {"f16": torch.float16, "bf16": torch.bfloat16, "f32": torch.float32}
 
 EXPORTS = ("ragged_pack", "ragged_attn_fwd", "ragged_unpack_cls", "ragged_unpack",
            "ragged_pipeline", "ragged_get_device_status", "ragged_status_string",
-           "ragged_last_error", "ragged_abi_version")
+           "ragged_last_error", "ragged_abi_version", "ragged_set_attn_kernel")
 
 
 class RaggedError(RuntimeError):
@@ -80,6 +84,8 @@ def load(path: Optional[str] = None):
     lib.ragged_last_error.restype = ctypes.c_char_p
     lib.ragged_abi_version.argtypes = []
     lib.ragged_abi_version.restype = ctypes.c_int32
+    lib.ragged_set_attn_kernel.argtypes = [ctypes.c_int32]
+    lib.ragged_set_attn_kernel.restype = ctypes.c_int32
     if path is None:
         _lib = lib
     return lib
@@ -113,6 +119,14 @@ def _dtype_code(t: torch.Tensor) -> int:
 
 def ragged_abi_version() -> int:
     return int(load().ragged_abi_version())
+
+
+def ragged_set_attn_kernel(kernel: int) -> int:
+    """Process-wide attention kernel choice (RAGGED_ATTN_*); returns the previous one."""
+    prev = int(load().ragged_set_attn_kernel(int(kernel)))
+    if prev < 0:
+        raise ValueError(f"unknown attention kernel {kernel}")
+    return prev
 
 
 def ragged_status_string(status: int) -> str:

@@ -1,0 +1,653 @@
+// Ragged bidirectional attention on the 5th-generation tensor cores
+// (tcgen05.mma with TMEM accumulators), f16 / bf16, head_dim 64.
+//
+// Operation ("Dispatch-Aware Ragged Attention for Pruned Vision Transformers",
+// abstract; radpulse section "Bypassing the binding"): per sequence b and head
+// h, O = softmax(scale Q K^T) V over the sequence's own rows.
+//
+// One CTA (4 warps) per (128-query tile, head, sequence), all of the
+// sequence's K and V resident in shared memory (up to 640 keys):
+//   - every load (Q tile, all K/V tiles) is issued at once with cp.async into
+//     128-byte-swizzled tiles, which are the canonical SWIZZLE_128B operand
+//     layouts of tcgen05 (K-major for Q, K and P; MN-major for V);
+//   - thread 0 issues S = Q K^T for each 64-key tile into TMEM as soon as
+//     that tile has landed (M = 128, N = 64, K = 64 in four K = 16 steps);
+//   - the softmax is one thread per query row (TMEM lane = row): the exact row
+//     maximum over all keys first, then p = exp2(s scale log2e - m) and the
+//     row sum, so the output never needs rescaling.  P is written to a
+//     double-buffered shared tile (bf16: split into bf16 hi + lo parts, each
+//     multiplied with V, so the product carries ~16 bits of P);
+//   - thread 0 accumulates O += P V into TMEM (N = 64 dims, K = 64 keys per
+//     tile), tcgen05.commit releasing each P buffer;
+//   - the epilogue reads O from TMEM, divides by the row sum and stores the
+//     row (and the CLS row).
+// S occupies TMEM columns [0, 448) and O columns [448, 512).  Sequences
+// longer than 448 keys take two passes over key chunks of 448: the first for
+// the row maxima, the second recomputes S for the probabilities.
+//
+// Every mbarrier wait is bounded; a wait that gives up sets
+// RAGGED_DEV_TIMEOUT in the status word and the CTA skips to its teardown
+// (TMEM is always freed).
+#pragma once
+
+#include "attn_resident.cuh"
+
+namespace ragged {
+namespace tc05 {
+
+using mma_attn::swz;
+using resident::PackedRows;
+
+constexpr int kThreads = 128;
+constexpr int kRows = 128;            // query rows per CTA (MMA M)
+constexpr int kTileN = 64;            // keys per tile
+constexpr int kChunkTiles = 7;        // key tiles per TMEM S chunk (448 columns)
+constexpr int kMaxTiles = 10;         // 640 keys resident
+constexpr int kMaxKeys = kMaxTiles * kTileN;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kOCol = kChunkTiles * kTileN;   // 448
+constexpr int kQBytes = kRows * 128;               // 16 KB
+constexpr int kKVTileBytes = kTileN * 128;         // 8 KB
+constexpr int kPTileBytes = kRows * 128;           // 16 KB (128 rows x 64 keys)
+constexpr int kMaxDynSmem = 230400;                // dynamic part, under the 227 KB per-block limit
+constexpr uint32_t kSpinLimit = 1u << 22;
+
+// Dynamic shared memory: 1 KB alignment slack, Q, K tiles, V tiles, P slots.
+__host__ __device__ constexpr int smem_bytes(int key_tiles, int p_slots, int p_parts) {
+    return 1024 + kQBytes + 2 * key_tiles * kKVTileBytes + p_slots * p_parts * kPTileBytes;
+}
+
+// ---- instruction and shared-memory descriptors -------------------------------
+
+// kind::f16 instruction descriptor: fp32 accumulate, A/B format (0 = f16,
+// 1 = bf16), A K-major, B K-major (0) or MN-major (1), M = 128, N.
+__device__ __forceinline__ uint32_t make_idesc(uint32_t ab_format, uint32_t b_mn_major, uint32_t n) {
+    return (1u << 4)                  // D format: f32
+           | (ab_format << 7)         // A format
+           | (ab_format << 10)        // B format
+           | (b_mn_major << 16)       // B major
+           | ((n >> 3) << 17)         // N / 8
+           | ((kRows >> 4) << 24);    // M / 16
+}
+
+// Shared-memory matrix descriptor for a 128-byte-swizzled tile whose 8-row
+// groups are 1024 bytes apart (both the K-major and the MN-major forms used
+// here); base must sit in a 1024-byte aligned atom.
+__device__ __forceinline__ uint64_t make_sdesc(uint32_t smem_byte_addr) {
+    return static_cast<uint64_t>((smem_byte_addr >> 4) & 0x3FFFu)     // start address
+           | (static_cast<uint64_t>(1) << 16)                          // leading byte offset (unused)
+           | (static_cast<uint64_t>(1024 >> 4) << 32)                  // stride byte offset
+           | (static_cast<uint64_t>(1) << 46)                          // descriptor version
+           | (static_cast<uint64_t>(2) << 61);                         // SWIZZLE_128B
+}
+
+// ---- tcgen05 / mbarrier wrappers -------------------------------------------
+
+__device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                        uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}\n"
+        :
+        : "r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(0), "r"(0), "r"(0), "r"(0)
+        : "memory");
+}
+
+__device__ __forceinline__ void mma_commit(uint32_t mbar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(mbar)
+                 : "memory");
+}
+
+__device__ __forceinline__ void fence_before_sync() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void fence_after_sync() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+__device__ __forceinline__ void mbar_init(uint32_t mbar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(mbar), "r"(count) : "memory");
+}
+
+// Waits for the phase with the given parity to complete; false after the
+// bounded number of polls.
+__device__ __forceinline__ bool mbar_wait(uint32_t mbar, uint32_t parity) {
+    for (uint32_t i = 0; i < kSpinLimit; ++i) {
+        uint32_t done;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}\n"
+            : "=r"(done)
+            : "r"(mbar), "r"(parity)
+            : "memory");
+        if (done) return true;
+    }
+    return false;
+}
+
+// 16 consecutive fp32 columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+    uint32_t r[16];
+    // The load and its wait sit in one statement so no use of r can be
+    // scheduled before the data has arrived.
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n\t"
+        "tcgen05.wait::ld.sync.aligned;\n"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr)
+        : "memory");
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Stores 16 consecutive fp32 columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};\n\t"
+        "tcgen05.wait::st.sync.aligned;\n"
+        :
+        : "r"(taddr), "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+          "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+          "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
+          "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+          "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+          "r"(__float_as_uint(v[15]))
+        : "memory");
+}
+
+// exp2 for the rescale factor; exp2(-inf) = 0 (a row with no reference yet).
+__device__ __forceinline__ float fast_exp2_guard(float x) { return mma_attn::fast_exp2(x); }
+
+template <typename T>
+struct Cvt;
+template <>
+struct Cvt<__half> {
+    static constexpr uint32_t kFormat = 0;
+    static constexpr int kParts = 1;
+    __device__ __forceinline__ static uint32_t pack(float lo, float hi) {
+        __half2 h = __floats2half2_rn(lo, hi);
+        return *reinterpret_cast<uint32_t*>(&h);
+    }
+};
+template <>
+struct Cvt<__nv_bfloat16> {
+    static constexpr uint32_t kFormat = 1;
+    static constexpr int kParts = 2;   // P = hi + lo
+    __device__ __forceinline__ static uint32_t pack(float lo, float hi) {
+        __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+        return *reinterpret_cast<uint32_t*>(&h);
+    }
+};
+
+template <typename T>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_tc05_kernel(PackedRows src, int key_tiles, int p_slots, float scale_log2, int H,
+                     uint16_t* __restrict__ out, int64_t out_tok_stride, uint16_t* __restrict__ cls_out) {
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ __align__(8) uint64_t s_mbar[4];   // 0: S ready, 1: O ready, 2, 3: P slot free
+    __shared__ uint32_t s_tmem;
+    __shared__ int s_fail;
+
+    const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    if (!src.begin(b, h, nullptr, nullptr)) return;
+    const int len = src.len, start = src.start;
+    const int q0 = qt * kRows;
+    if (q0 >= len) return;
+    const int nt = (len + kTileN - 1) / kTileN;
+    const int tid = threadIdx.x, warp = tid >> 5;
+    constexpr int kParts = Cvt<T>::kParts;
+
+    const uint32_t raw = smem_addr(smem_raw);
+    const uint32_t sQ = (raw + 1023u) & ~1023u;
+    const uint32_t sK = sQ + kQBytes;
+    const uint32_t sV = sK + key_tiles * kKVTileBytes;
+    const uint32_t sP = sV + key_tiles * kKVTileBytes;
+    const uint32_t slot_bytes = kParts * kPTileBytes;
+    uint8_t* gP = smem_raw + (sP - raw);
+
+    // Loads: group 0 = Q + key tile 0, group t = key tile t.
+    resident::load_tile<kRows>(sQ, src, 0, q0, len);
+    for (int t = 0; t < nt; ++t) {
+        resident::load_tile<kTileN>(sK + t * kKVTileBytes, src, 1, t * kTileN, len);
+        resident::load_tile<kTileN>(sV + t * kKVTileBytes, src, 2, t * kTileN, len);
+        cp_async_commit();
+    }
+
+    const uint32_t mbar0 = smem_addr(&s_mbar[0]);
+    if (tid == 0) {
+        for (int i = 0; i < 4; ++i) mbar_init(mbar0 + 8 * i, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        s_fail = 0;
+    }
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(&s_tmem)),
+                     "r"(kTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tmem = s_tmem;
+    const uint32_t t_lane = tmem + (static_cast<uint32_t>(warp * 32) << 16);   // this warp's TMEM lanes
+
+    const uint32_t idesc_qk = make_idesc(Cvt<T>::kFormat, 0, kTileN);
+    const uint32_t idesc_pv = make_idesc(Cvt<T>::kFormat, 1, 64);
+    const int row = q0 + tid;               // this thread's query row (TMEM lane = tid)
+    const int nchunks = (nt + kChunkTiles - 1) / kChunkTiles;
+    uint32_t s_phase = 0;
+    uint32_t p_phase[2] = {0, 0};
+    float m = -INFINITY, l = 0.f;
+
+    // S = Q K^T for the tiles of one chunk, issued tile by tile; when
+    // wait_loads, each tile's cp.async group is awaited first (first pass).
+    auto issue_chunk = [&](int c, bool wait_loads) {
+        const int t0 = c * kChunkTiles, t1 = min(nt, t0 + kChunkTiles);
+        for (int t = t0; t < t1; ++t) {
+            if (wait_loads) {
+                resident::cp_async_wait_pending(nt - 1 - t);
+                fence_async_smem();
+            }
+            fence_before_sync();
+            __syncthreads();
+            if (tid == 0) {
+                fence_after_sync();
+                const uint32_t d = tmem + static_cast<uint32_t>((t - t0) * kTileN);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_f16(d, make_sdesc(sQ + ks * 32), make_sdesc(sK + t * kKVTileBytes + ks * 32), idesc_qk,
+                            ks > 0);
+            }
+        }
+        if (tid == 0) mma_commit(mbar0);
+        if (!mbar_wait(mbar0, s_phase)) atomicExch(&s_fail, 1);
+        s_phase ^= 1;
+        fence_after_sync();
+    };
+
+    // ---- pass 1: exact row maxima over all keys ----
+    for (int c = 0; c < nchunks; ++c) {
+        if (c > 0) {   // the previous chunk's S must be fully read before it is overwritten
+            fence_before_sync();
+            __syncthreads();
+        }
+        issue_chunk(c, c == 0);
+        if (c == 0 && nchunks > 1) {   // later chunks' loads are awaited here once
+            resident::cp_async_wait_pending(0);
+            fence_async_smem();
+        }
+        const int t0 = c * kChunkTiles, t1 = min(nt, t0 + kChunkTiles);
+        for (int t = t0; t < t1; ++t) {
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+                float v[16];
+                tmem_ld16(t_lane + static_cast<uint32_t>((t - t0) * kTileN + g * 16), v);
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    if (t * kTileN + g * 16 + i < len) m = fmaxf(m, v[i]);
+            }
+        }
+    }
+    const float mb = m * scale_log2;
+
+    // ---- pass 2: probabilities, P V ----
+    for (int c = 0; c < nchunks; ++c) {
+        if (nchunks > 1) {
+            fence_before_sync();
+            __syncthreads();
+            issue_chunk(c, false);
+        }
+        if (s_fail) break;
+        const int t0 = c * kChunkTiles, t1 = min(nt, t0 + kChunkTiles);
+        for (int t = t0; t < t1; ++t) {
+            const int slot = p_slots == 2 ? (t & 1) : 0;
+            if (t >= p_slots) {   // the P V product of tile t - p_slots has released this slot
+                if (!mbar_wait(mbar0 + 16 + 8 * slot, p_phase[slot])) atomicExch(&s_fail, 1);
+                p_phase[slot] ^= 1;
+            }
+            uint8_t* p_hi = gP + slot * slot_bytes;
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+                float v[16];
+                tmem_ld16(t_lane + static_cast<uint32_t>((t - t0) * kTileN + g * 16), v);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const bool ok = t * kTileN + g * 16 + i < len;
+                    v[i] = ok ? mma_attn::fast_exp2(fmaf(v[i], scale_log2, -mb)) : 0.f;
+                    l += v[i];
+                }
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    uint32_t w[4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) w[i] = Cvt<T>::pack(v[half * 8 + 2 * i], v[half * 8 + 2 * i + 1]);
+                    const int chunk = g * 2 + half;
+                    *reinterpret_cast<uint4*>(p_hi + swz(tid, chunk)) = make_uint4(w[0], w[1], w[2], w[3]);
+                    if constexpr (kParts == 2) {
+                        uint32_t r[4];
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            __nv_bfloat162 hb = *reinterpret_cast<__nv_bfloat162*>(&w[i]);
+                            const float2 f = __bfloat1622float2(hb);
+                            r[i] = Cvt<T>::pack(v[half * 8 + 2 * i] - f.x, v[half * 8 + 2 * i + 1] - f.y);
+                        }
+                        *reinterpret_cast<uint4*>(p_hi + kPTileBytes + swz(tid, chunk)) =
+                            make_uint4(r[0], r[1], r[2], r[3]);
+                    }
+                }
+            }
+            fence_async_smem();
+            fence_before_sync();
+            __syncthreads();
+            if (s_fail) break;
+            if (tid == 0) {
+                fence_after_sync();
+                const uint32_t p_addr = sP + slot * slot_bytes;
+#pragma unroll
+                for (int part = 0; part < kParts; ++part)
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)
+                        mma_f16(tmem + kOCol, make_sdesc(p_addr + part * kPTileBytes + ks * 32),
+                                make_sdesc(sV + t * kKVTileBytes + ks * 2048), idesc_pv,
+                                (t > 0 || part > 0 || ks > 0) ? 1u : 0u);
+                mma_commit(mbar0 + 16 + 8 * slot);
+            }
+        }
+    }
+
+    // ---- epilogue: O / l ----
+    if (tid == 0 && !s_fail) mma_commit(mbar0 + 8);
+    __syncthreads();
+    if (!s_fail) {
+        if (!mbar_wait(mbar0 + 8, 0)) {
+            atomicExch(&s_fail, 1);
+        } else {
+            fence_after_sync();
+            const float inv = 1.f / l;
+            uint32_t w[32];
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+                float v[16];
+                tmem_ld16(t_lane + kOCol + g * 16, v);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) w[g * 8 + i] = Cvt<T>::pack(v[2 * i] * inv, v[2 * i + 1] * inv);
+            }
+            if (row < len) {
+                uint4* dst = reinterpret_cast<uint4*>(out + static_cast<int64_t>(start + row) * out_tok_stride +
+                                                      h * 64);
+#pragma unroll
+                for (int c = 0; c < 8; ++c) dst[c] = make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+                if (row == 0 && cls_out != nullptr) {
+                    uint4* cd = reinterpret_cast<uint4*>(cls_out + (static_cast<int64_t>(b) * H + h) * 64);
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) cd[c] = make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+                }
+            }
+        }
+    }
+
+    // ---- teardown: loads drained, TMEM freed ----
+    resident::cp_async_wait_pending(0);
+    fence_before_sync();
+    __syncthreads();
+    if (s_fail && tid == 0) raise_status(RAGGED_DEV_TIMEOUT);
+    if (warp == 0) {
+        fence_after_sync();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
+    }
+}
+
+
+// ---------------------------------------------------------------------------
+// Streaming variant: two CTAs per SM.
+//
+// Same operation and roles as attn_tc05_kernel, but the K/V tiles of a
+// sequence flow through a 3-stage shared-memory ring (loads run two tiles
+// ahead) and TMEM holds only two 64-column S buffers and O (256 columns), so
+// two CTAs share each SM and one's softmax overlaps the other's loads and
+// MMAs.  Within a CTA, S = Q K^T of tile t + 1 is issued before the softmax of
+// tile t.  The softmax is single-pass: each row keeps a reference maximum and
+// rescales its running sum and O (in TMEM) only when a tile raises the row
+// maximum by more than 2^8 in base 2; otherwise the probabilities
+// exp2(s - reference) stay below 256 and the reference is kept.  The final
+// division by the running sum makes the result independent of the reference.
+// ---------------------------------------------------------------------------
+
+constexpr uint32_t kStreamTmemCols = 256;
+constexpr uint32_t kStreamOCol = 128;          // S buffers at columns 0 and 64
+constexpr int kStages = 3;
+constexpr float kRescaleThreshold = 8.f;       // log2 units
+
+__host__ __device__ constexpr int stream_smem_bytes(int p_parts) {
+    // alignment slack, Q, K/V ring, P (two slots for f16, one hi/lo pair for bf16)
+    return 1024 + kQBytes + kStages * 2 * kKVTileBytes + 2 * kPTileBytes;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kThreads, 2)
+    attn_tc05_stream_kernel(PackedRows src, float scale_log2, int H, uint16_t* __restrict__ out,
+                            int64_t out_tok_stride, uint16_t* __restrict__ cls_out) {
+    extern __shared__ uint8_t smem_raw[];
+    // mbarriers: 0, 1: S buffer ready; 2, 3: P V product of slot done
+    __shared__ __align__(8) uint64_t s_mbar[4];
+    __shared__ uint32_t s_tmem;
+    __shared__ int s_fail;
+
+    const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    if (!src.begin(b, h, nullptr, nullptr)) return;
+    const int len = src.len, start = src.start;
+    const int q0 = qt * kRows;
+    if (q0 >= len) return;
+    const int nt = (len + kTileN - 1) / kTileN;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    constexpr int kParts = Cvt<T>::kParts;
+    constexpr int kSlots = 2 / kParts;     // f16: two P slots; bf16: one hi/lo pair
+
+    const uint32_t raw = smem_addr(smem_raw);
+    const uint32_t sQ = (raw + 1023u) & ~1023u;
+    const uint32_t sRing = sQ + kQBytes;                         // stage s: K at +s*16K, V at +8K
+    const uint32_t sP = sRing + kStages * 2 * kKVTileBytes;
+    uint8_t* gP = smem_raw + (sP - raw);
+    auto stage_k = [&](int t) { return sRing + (t % kStages) * 2 * kKVTileBytes; };
+    auto stage_v = [&](int t) { return stage_k(t) + kKVTileBytes; };
+    auto load_kv = [&](int t) {
+        resident::load_tile<kTileN>(stage_k(t), src, 1, t * kTileN, len);
+        resident::load_tile<kTileN>(stage_v(t), src, 2, t * kTileN, len);
+        cp_async_commit();
+    };
+
+    // Loads: group 0 = Q + tile 0, then one group per tile, two tiles ahead.
+    resident::load_tile<kRows>(sQ, src, 0, q0, len);
+    load_kv(0);
+    if (nt > 1) load_kv(1);
+
+    const uint32_t mbar0 = smem_addr(&s_mbar[0]);
+    if (tid == 0) {
+        for (int i = 0; i < 4; ++i) mbar_init(mbar0 + 8 * i, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        s_fail = 0;
+    }
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(&s_tmem)),
+                     "r"(kStreamTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tmem = s_tmem;
+    const uint32_t t_lane = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+
+    const uint32_t idesc_qk = make_idesc(Cvt<T>::kFormat, 0, kTileN);
+    const uint32_t idesc_pv = make_idesc(Cvt<T>::kFormat, 1, 64);
+    const int row = q0 + tid;
+
+    // Waits until this thread's copies of tile t have landed, leaving
+    // `pending` later groups in flight, and publishes them to the tensor core;
+    // includes the CTA barrier.
+    auto tile_landed = [&](int pending) {
+        if (pending) cp_async_wait<1>(); else cp_async_wait<0>();
+        fence_async_smem();
+        fence_before_sync();
+        __syncthreads();
+    };
+    auto issue_qk = [&](int t) {   // by thread 0, after tile t has landed
+        fence_after_sync();
+        const uint32_t d = tmem + static_cast<uint32_t>((t & 1) * kTileN);
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+            mma_f16(d, make_sdesc(sQ + ks * 32), make_sdesc(stage_k(t) + ks * 32), idesc_qk, ks > 0);
+        mma_commit(mbar0 + 8 * (t & 1));
+    };
+    // mbarrier k (k = 0, 1) completes once per tile t with t % 2 == k, so the
+    // wait for tile t uses parity (t / 2) & 1.
+    auto wait_tile_event = [&](uint32_t mbar, int t) {
+        if (!mbar_wait(mbar, static_cast<uint32_t>((t >> 1) & 1))) atomicExch(&s_fail, 1);
+    };
+
+    tile_landed(nt > 1 ? 1 : 0);
+    if (tid == 0) issue_qk(0);
+
+    float m_ref = -INFINITY;   // reference maximum (log2 units) of this row
+    float l = 0.f;
+    for (int t = 0; t < nt; ++t) {
+        // (a) S of tile t + 1 (landed: issued one iteration ago) is computed
+        // while this tile's softmax runs; its S buffer was last read by the
+        // softmax of tile t - 1, which is finished.
+        if (t + 1 < nt) {
+            tile_landed(0);
+            if (s_fail) break;
+            if (tid == 0) issue_qk(t + 1);
+        }
+        // (b) Once the product of tile t - 1 is done (and with it every earlier
+        // product, so both P slots and the stage of tile t - 1 are free),
+        // refill that stage with tile t + 2.
+        if (t >= 1) wait_tile_event(mbar0 + 16 + 8 * ((t - 1) & 1), t - 1);
+        if (t + 2 < nt) load_kv(t + 2);
+        // (c) S of tile t.
+        wait_tile_event(mbar0 + 8 * (t & 1), t);
+        fence_after_sync();
+
+        float sv[4][16];
+        float mt = -INFINITY;
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+            tmem_ld16(t_lane + static_cast<uint32_t>((t & 1) * kTileN + g * 16), sv[g]);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const bool ok = t * kTileN + g * 16 + i < len;
+                sv[g][i] = ok ? sv[g][i] * scale_log2 : -INFINITY;
+                mt = fmaxf(mt, sv[g][i]);
+            }
+        }
+        // (d) Rescale only when the tile's maximum exceeds the reference by
+        // more than the threshold (always for the first tile).
+        const bool grow = mt > m_ref + kRescaleThreshold;
+        float alpha = 1.f;
+        if (grow) {
+            alpha = fast_exp2_guard(m_ref - mt);
+            l *= alpha;
+            m_ref = mt;
+        }
+        if (t > 0 && __any_sync(0xffffffffu, grow)) {
+            // O holds the (finished, see (b)) products of tiles 0 .. t - 1:
+            // scale this warp's rows in TMEM; rows that keep their reference
+            // are multiplied by 1.
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+                float ov[16];
+                tmem_ld16(t_lane + kStreamOCol + g * 16, ov);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) ov[i] *= alpha;
+                tmem_st16(t_lane + kStreamOCol + g * 16, ov);
+            }
+        }
+
+        uint8_t* p_base = gP + (kSlots == 2 ? (t & 1) : 0) * kPTileBytes;
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                sv[g][i] = mma_attn::fast_exp2(sv[g][i] - m_ref);   // -inf -> 0
+                l += sv[g][i];
+            }
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                uint32_t w[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) w[i] = Cvt<T>::pack(sv[g][half * 8 + 2 * i], sv[g][half * 8 + 2 * i + 1]);
+                const int chunk = g * 2 + half;
+                *reinterpret_cast<uint4*>(p_base + swz(tid, chunk)) = make_uint4(w[0], w[1], w[2], w[3]);
+                if constexpr (kParts == 2) {
+                    uint32_t r[4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        __nv_bfloat162 hb = *reinterpret_cast<__nv_bfloat162*>(&w[i]);
+                        const float2 f = __bfloat1622float2(hb);
+                        r[i] = Cvt<T>::pack(sv[g][half * 8 + 2 * i] - f.x, sv[g][half * 8 + 2 * i + 1] - f.y);
+                    }
+                    *reinterpret_cast<uint4*>(p_base + kPTileBytes + swz(tid, chunk)) =
+                        make_uint4(r[0], r[1], r[2], r[3]);
+                }
+            }
+        }
+        fence_async_smem();
+        fence_before_sync();
+        __syncthreads();
+        if (s_fail) break;
+        if (tid == 0) {
+            fence_after_sync();
+            const uint32_t p_addr = sP + (kSlots == 2 ? (t & 1) : 0) * kPTileBytes;
+#pragma unroll
+            for (int part = 0; part < kParts; ++part)
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_f16(tmem + kStreamOCol, make_sdesc(p_addr + part * kPTileBytes + ks * 32),
+                            make_sdesc(stage_v(t) + ks * 2048), idesc_pv, (t > 0 || part > 0 || ks > 0) ? 1u : 0u);
+            mma_commit(mbar0 + 16 + 8 * (t & 1));
+        }
+    }
+
+    // Epilogue: wait for the last product, O / l.
+    if (!s_fail) {
+        wait_tile_event(mbar0 + 16 + 8 * ((nt - 1) & 1), nt - 1);
+        if (!s_fail) {
+            fence_after_sync();
+            const float inv = 1.f / l;
+            uint32_t w[32];
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+                float v[16];
+                tmem_ld16(t_lane + kStreamOCol + g * 16, v);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) w[g * 8 + i] = Cvt<T>::pack(v[2 * i] * inv, v[2 * i + 1] * inv);
+            }
+            if (row < len) {
+                uint4* dst = reinterpret_cast<uint4*>(out + static_cast<int64_t>(start + row) * out_tok_stride +
+                                                      h * 64);
+#pragma unroll
+                for (int c = 0; c < 8; ++c) dst[c] = make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+                if (row == 0 && cls_out != nullptr) {
+                    uint4* cd = reinterpret_cast<uint4*>(cls_out + (static_cast<int64_t>(b) * H + h) * 64);
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) cd[c] = make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+                }
+            }
+        }
+    }
+
+    cp_async_wait<0>();
+    fence_before_sync();
+    __syncthreads();
+    if (s_fail && tid == 0) raise_status(RAGGED_DEV_TIMEOUT);
+    if (warp == 0) {
+        fence_after_sync();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kStreamTmemCols)
+                     : "memory");
+    }
+    (void)lane;
+}
+
+}  // namespace tc05
+}  // namespace ragged

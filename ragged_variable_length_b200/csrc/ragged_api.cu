@@ -12,6 +12,8 @@
 #include "attn_f32.cuh"
 #include "attn_mma.cuh"
 #include "attn_resident.cuh"
+#include "attn_tc05.cuh"
+#include <atomic>
 #include "common.cuh"
 #include "pack.cuh"
 
@@ -133,6 +135,24 @@ ragged_status launch_resident_ks(const Src& src, int64_t B, int64_t H, int key_t
     return cuda_check(cudaGetLastError(), "resident attention launch");
 }
 
+std::atomic<int> g_attn_kernel{RAGGED_ATTN_AUTO};
+bool g_tc05_smem[2][kMaxDevices];
+
+template <typename T>
+ragged_status launch_tc05(const ragged::resident::PackedRows& src, int64_t B, int64_t H, int64_t max_seqlen,
+                          float scale, void* out, int64_t out_tok_stride, void* cls_out, int slot, cudaStream_t s) {
+    using namespace ragged::tc05;
+    auto kernel = attn_tc05_stream_kernel<T>;
+    const int smem = stream_smem_bytes(std::is_same<T, __nv_bfloat16>::value ? 2 : 1);
+    ragged_status st = ensure_smem(kernel, smem, g_tc05_smem[slot]);
+    if (st != RAGGED_OK) return st;
+    const dim3 grid(static_cast<unsigned>((max_seqlen + kRows - 1) / kRows), static_cast<unsigned>(H),
+                    static_cast<unsigned>(B));
+    kernel<<<grid, kThreads, smem, s>>>(src, scale * 1.4426950408889634f, static_cast<int>(H),
+                                        static_cast<uint16_t*>(out), out_tok_stride, static_cast<uint16_t*>(cls_out));
+    return cuda_check(cudaGetLastError(), "tcgen05 attention launch");
+}
+
 // slot: 0/1 packed f16/bf16, 2/3 dense f16/bf16 (one set of smem flags per kernel).
 bool g_res_smem_ks[4][3][kMaxDevices];
 
@@ -158,6 +178,11 @@ ragged_status launch_resident(const Src& src, int64_t B, int64_t H, int key_tile
 extern "C" {
 
 int32_t ragged_abi_version(void) { return kAbiVersion; }
+
+int32_t ragged_set_attn_kernel(int32_t kernel) {
+    if (kernel < RAGGED_ATTN_AUTO || kernel > RAGGED_ATTN_TCGEN05) return -1;
+    return g_attn_kernel.exchange(kernel);
+}
 
 const char* ragged_last_error(void) { return g_last_error; }
 
@@ -278,19 +303,30 @@ ragged_status ragged_attn_fwd(const void* q, const void* k, const void* v, int64
             static_cast<float*>(out), out_tok_stride, static_cast<float*>(cls_out));
         return cuda_check(cudaGetLastError(), "attention (f32) launch");
     }
-    // Whole-sequence residency pays off in the latency-bound regime (few CTAs:
-    // keys split across warps) and for single-tile sequences; large launches
-    // of longer sequences keep more CTAs per SM with the streaming kernel.
+    // Kernel choice.  AUTO: whole-sequence residency pays off in the
+    // latency-bound regime (few CTAs: keys split across warps) and for
+    // single-tile sequences; other launches stream K/V tiles.
     const int res_tiles = static_cast<int>((max_seqlen + 63) / 64);
-    if (max_seqlen <= ragged::resident::kMaxKeys &&
-        (res_tiles == 1 || resident_ksplit(B, H, res_tiles) > 1)) {
-        ragged::resident::PackedRows src{static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(k),
-                                         static_cast<const uint16_t*>(v), tok_stride, head_stride, cu_seqlens,
-                                         static_cast<int>(max_seqlen), 0, 0, 0};
-        const int key_tiles = static_cast<int>((max_seqlen + 63) / 64);
+    int kernel_choice = g_attn_kernel.load(std::memory_order_relaxed);
+    if (kernel_choice == RAGGED_ATTN_AUTO)
+        kernel_choice = (max_seqlen <= ragged::resident::kMaxKeys &&
+                         (res_tiles == 1 || resident_ksplit(B, H, res_tiles) > 1))
+                            ? RAGGED_ATTN_RESIDENT
+                            : RAGGED_ATTN_STREAMING;
+    if (kernel_choice == RAGGED_ATTN_RESIDENT && max_seqlen > ragged::resident::kMaxKeys)
+        return fail(RAGGED_ERR_UNSUPPORTED, "the resident attention kernel holds at most 640 keys");
+    ragged::resident::PackedRows src{static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(k),
+                                     static_cast<const uint16_t*>(v), tok_stride, head_stride, cu_seqlens,
+                                     static_cast<int>(max_seqlen), 0, 0, 0};
+    if (kernel_choice == RAGGED_ATTN_TCGEN05) {
         if (dtype == RAGGED_F16)
-            return launch_resident<__half>(src, B, H, key_tiles, 0, scale, out, out_tok_stride, cls_out, nullptr, 0, s);
-        return launch_resident<__nv_bfloat16>(src, B, H, key_tiles, 0, scale, out, out_tok_stride, cls_out, nullptr,
+            return launch_tc05<__half>(src, B, H, max_seqlen, scale, out, out_tok_stride, cls_out, 0, s);
+        return launch_tc05<__nv_bfloat16>(src, B, H, max_seqlen, scale, out, out_tok_stride, cls_out, 1, s);
+    }
+    if (kernel_choice == RAGGED_ATTN_RESIDENT) {
+        if (dtype == RAGGED_F16)
+            return launch_resident<__half>(src, B, H, res_tiles, 0, scale, out, out_tok_stride, cls_out, nullptr, 0, s);
+        return launch_resident<__nv_bfloat16>(src, B, H, res_tiles, 0, scale, out, out_tok_stride, cls_out, nullptr,
                                               1, s);
     }
     using namespace ragged::mma_attn;

@@ -18,11 +18,13 @@ from helpers import TORCH_DTYPE, attn_error, to_device, to_f64
 pytestmark = pytest.mark.gpu
 
 
-def run_pipeline(w, separate_qkv=False, out_pad=0, max_seqlen=None):
-    """Device pack -> attend (with fused CLS) for a synthetic workload.
+KERNELS = {"auto": rv.RAGGED_ATTN_AUTO, "streaming": rv.RAGGED_ATTN_STREAMING,
+           "resident": rv.RAGGED_ATTN_RESIDENT, "tcgen05": rv.RAGGED_ATTN_TCGEN05}
 
-    max_seqlen above 640 selects the streaming attention kernel; the default
-    (L_full) selects the resident one when L_full <= 640."""
+
+def run_pipeline(w, separate_qkv=False, out_pad=0, max_seqlen=None, kernel="auto"):
+    """Device pack -> attend (with fused CLS) for a synthetic workload, with
+    the given attention kernel (the fp32 check path has a single kernel)."""
     dense = to_device(w.qkv, w.dtype)
     keep = torch.from_numpy(w.keep).cuda()
     packed, cu = rv.ragged_pack(dense, keep)
@@ -35,7 +37,11 @@ def run_pipeline(w, separate_qkv=False, out_pad=0, max_seqlen=None):
         q, k, v = (packed[:, i].contiguous() for i in range(3))
     else:
         q, k, v = packed[:, 0], packed[:, 1], packed[:, 2]
-    rv.ragged_attn_fwd(q, k, v, cu, max_seqlen or w.L_full, w.scale, out=out, cls_out=cls)
+    prev = rv.ragged_set_attn_kernel(KERNELS[kernel])
+    try:
+        rv.ragged_attn_fwd(q, k, v, cu, max_seqlen or w.L_full, w.scale, out=out, cls_out=cls)
+    finally:
+        rv.ragged_set_attn_kernel(prev)
     torch.cuda.synchronize()
     assert rv.ragged_get_device_status() == 0
     return cu.cpu().numpy(), out, cls, out_full
@@ -68,17 +74,27 @@ def check_against_oracle(w, seqs=None, **kw):
     return err
 
 
-@pytest.mark.parametrize("dtype", ["f16", "bf16", "f32"])
-def test_tiny_all_elements(dtype):
-    check_against_oracle(synthetic.tiny(dtype))
+KERNEL_CASES = [("f16", k) for k in KERNELS] + [("bf16", k) for k in KERNELS] + [("f32", "auto")]
 
 
-@pytest.mark.parametrize("dtype", ["f16", "bf16", "f32"])
-@pytest.mark.parametrize("kernel", ["resident", "streaming"])
+@pytest.mark.parametrize("dtype,kernel", KERNEL_CASES)
+def test_tiny_all_elements(dtype, kernel):
+    check_against_oracle(synthetic.tiny(dtype), kernel=kernel)
+
+
+@pytest.mark.parametrize("dtype,kernel", KERNEL_CASES)
 def test_tile_edge_lengths(dtype, kernel):
     lengths = [1, 2, 15, 16, 17, 31, 32, 33, 63, 64, 65, 127, 128, 129, 191, 192, 193, 200]
     w = synthetic.make_workload("edges", len(lengths), 200, 3, lengths, dtype, 77)
-    check_against_oracle(w, max_seqlen=None if kernel == "resident" else 1000)
+    check_against_oracle(w, kernel=kernel)
+
+
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+def test_streaming_kernel_under_a_loose_bound(dtype):
+    """A max_seqlen far above the longest sequence only sizes the launch."""
+    lengths = [1, 2, 63, 64, 65, 128, 129, 200]
+    w = synthetic.make_workload("edges_loose", len(lengths), 200, 3, lengths, dtype, 76)
+    check_against_oracle(w, max_seqlen=1000)
 
 
 @pytest.mark.parametrize("dtype", ["f16", "bf16"])
@@ -88,22 +104,45 @@ def test_long_sequences_streaming_kernel(dtype):
     check_against_oracle(w)
 
 
-def test_resident_and_streaming_agree_with_the_bound_unused():
-    """A larger max_seqlen than needed changes the kernel, not the result's accuracy."""
-    w = synthetic.deit_b_pruned80()
-    a = check_against_oracle(w)
-    b = check_against_oracle(w, max_seqlen=2000)
-    assert a < 4e-3 and b < 4e-3
+def test_kernel_limits_are_reported():
+    """The kernel that holds whole sequences refuses launches longer than 640 keys."""
+    w = synthetic.make_workload("too_long", 1, 700, 1, [700], "f16", 82)
+    with pytest.raises(rv.RaggedError, match="640"):
+        run_pipeline(w, kernel="resident")
+
+
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+def test_long_sequences_tcgen05(dtype):
+    """The tcgen05 kernel streams K/V, so it takes sequences of any length."""
+    w = synthetic.make_workload("long_tc", 4, 1000, 2, [1000, 700, 641, 65], dtype, 83)
+    check_against_oracle(w, kernel="tcgen05")
+
+
+def test_tcgen05_rescale_path():
+    """Keys whose logits jump by far more than the rescale threshold after the
+    first tile force the in-TMEM rescaling of O."""
+    w = synthetic.make_workload("jump", 3, 300, 2, [300, 200, 129], "f16", 84)
+    q = w.qkv[:, :, 0].astype(np.float32)
+    k = w.qkv[:, :, 1].astype(np.float32)
+    k[:, 150:, :, :] = (k[:, 150:, :, :] * 6.0)          # later keys: logits up to ~6x larger
+    q *= 2.0
+    w.qkv = w.qkv.copy()
+    w.qkv[:, :, 0] = q.astype(np.float16)
+    w.qkv[:, :, 1] = k.astype(np.float16)
+    check_against_oracle(w, kernel="tcgen05")
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "f16"])
-def test_hires_lengths_576_577_640(dtype):
-    w = synthetic.make_workload("hires_edges", 4, 640, 2, [577, 576, 300, 640], dtype, 78)
-    check_against_oracle(w)
+@pytest.mark.parametrize("kernel", list(KERNELS))
+def test_hires_lengths_448_449_576_577_640(dtype, kernel):
+    """Around the tcgen05 kernel's single-pass limit (448 keys) and the resident limit (640)."""
+    w = synthetic.make_workload("hires_edges", 6, 640, 2, [577, 576, 300, 640, 448, 449], dtype, 78)
+    check_against_oracle(w, kernel=kernel)
 
 
-def test_deit_b_pruned80_all_sequences():
-    check_against_oracle(synthetic.deit_b_pruned80())
+@pytest.mark.parametrize("kernel", list(KERNELS))
+def test_deit_b_pruned80_all_sequences(kernel):
+    check_against_oracle(synthetic.deit_b_pruned80(), kernel=kernel)
 
 
 @pytest.mark.parametrize("B", synthetic.SERVING_BATCHES)
@@ -112,41 +151,47 @@ def test_serving_all_sequences(B, rate):
     check_against_oracle(synthetic.serving(B, rate))
 
 
-@pytest.mark.parametrize("kernel", ["resident", "streaming"])
+@pytest.mark.parametrize("kernel", list(KERNELS))
 def test_hires_384_sampled(kernel):
     w = synthetic.hires_384()
-    check_against_oracle(w, seqs=sample_sequences(w.lengths, 6), max_seqlen=None if kernel == "resident" else 1024)
+    check_against_oracle(w, seqs=sample_sequences(w.lengths, 6), kernel=kernel)
 
 
 @pytest.mark.parametrize("rate", [0.0, 0.5, 0.9])
-def test_sweep_b512_sampled(rate):
+@pytest.mark.parametrize("kernel", list(KERNELS))
+def test_sweep_b512_sampled(rate, kernel):
     w = synthetic.sweep(rate)
-    check_against_oracle(w, seqs=sample_sequences(w.lengths, 8, seed=int(rate * 10)))
+    check_against_oracle(w, seqs=sample_sequences(w.lengths, 8, seed=int(rate * 10)), kernel=kernel)
 
 
-@pytest.mark.parametrize("dtype", ["f16", "bf16", "f32"])
-def test_separate_qkv_and_padded_output_rows(dtype):
+@pytest.mark.parametrize("dtype,kernel", KERNEL_CASES)
+def test_separate_qkv_and_padded_output_rows(dtype, kernel):
     w = synthetic.make_workload("layout", 5, 130, 4, [130, 1, 64, 65, 99], dtype, 79)
-    check_against_oracle(w, separate_qkv=True, out_pad=64 if dtype != "f32" else 32)
+    check_against_oracle(w, separate_qkv=True, out_pad=64 if dtype != "f32" else 32, kernel=kernel)
 
 
-@pytest.mark.parametrize("dtype", ["f16", "bf16", "f32"])
-def test_deterministic(dtype):
+@pytest.mark.parametrize("dtype,kernel", KERNEL_CASES)
+def test_deterministic(dtype, kernel):
     w = synthetic.make_workload("det", 6, 197, 6, [197, 40, 88, 3, 150, 64], dtype, 80)
-    _, out1, cls1, _ = run_pipeline(w)
-    _, out2, cls2, _ = run_pipeline(w)
+    _, out1, cls1, _ = run_pipeline(w, kernel=kernel)
+    _, out2, cls2, _ = run_pipeline(w, kernel=kernel)
     T = int(w.lengths.sum())
     assert torch.equal(out1[:T], out2[:T]) and torch.equal(cls1, cls2)
 
 
-def test_bad_cu_seqlens_are_flagged_and_skipped():
+@pytest.mark.parametrize("kernel", list(KERNELS))
+def test_bad_cu_seqlens_are_flagged_and_skipped(kernel):
     H, d = 2, 64
     q = torch.randn(100, H, d, device="cuda", dtype=torch.float16)
     out = torch.full((100, H, d), 7.0, dtype=torch.float16, device="cuda")
     rv.ragged_get_device_status()
     # sequence 0 is longer than the host bound; sequence 1 has a negative length
     cu = torch.tensor([0, 80, 60], dtype=torch.int32, device="cuda")
-    rv.ragged_attn_fwd(q, q, q, cu, max_seqlen=64, out=out)
+    prev = rv.ragged_set_attn_kernel(KERNELS[kernel])
+    try:
+        rv.ragged_attn_fwd(q, q, q, cu, max_seqlen=64, out=out)
+    finally:
+        rv.ragged_set_attn_kernel(prev)
     assert rv.ragged_get_device_status() & rv.RAGGED_DEV_BAD_SEQLENS
     assert torch.all(out == 7.0)
     assert rv.ragged_get_device_status() == 0     # reading clears the word
