@@ -19,7 +19,8 @@
  *    keeps no pointer after returning.
  *  - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
  *    stream).  Work is only enqueued: no call synchronises with the device,
- *    except ragged_get_device_status, which says so.
+ *    except ragged_get_device_status and ragged_pipeline with
+ *    RAGGED_PIPELINE_SYNC, which say so.
  *  - Every call returns a ragged_status.  Argument errors are detected on the
  *    host before anything is enqueued; nothing is launched then and
  *    ragged_last_error() describes the problem.  A launch failure reported by
@@ -191,6 +192,7 @@ RAGGED_API ragged_status ragged_unpack(const void *packed, const int32_t *cu_seq
 #define RAGGED_PIPELINE_AUTO 0u  /* choose per shape (see below)                  */
 #define RAGGED_PIPELINE_FUSED 1u /* one launch: pack, attention and CLS together    */
 #define RAGGED_PIPELINE_SPLIT 2u /* two launches: ragged_pack, then ragged_attn_fwd */
+#define RAGGED_PIPELINE_SYNC 4u  /* return after the work has finished on `stream`  */
 
 /*
  * ragged_pipeline - pack -> attend -> CLS in one host call.
@@ -213,6 +215,12 @@ RAGGED_API ragged_status ragged_unpack(const void *packed, const int32_t *cu_seq
  * the images before its own stays cheap; otherwise the split mode.  Results
  * are identical in both modes.  Requirements as for ragged_pack and
  * ragged_attn_fwd, with max_seqlen = L_full and scale positive and finite.
+ *
+ * RAGGED_PIPELINE_SYNC (may be combined with either mode) makes the call wait
+ * for the enqueued work (cudaStreamSynchronize on `stream`) before returning,
+ * for callers that want the results on return without a second call; it is
+ * the only form of any entry point besides ragged_get_device_status that
+ * synchronises, and it must not be used during stream capture.
  */
 RAGGED_API ragged_status ragged_pipeline(const void *dense_qkv, const uint8_t *keep, int64_t B,
                                          int64_t L_full, int64_t H, int64_t head_dim, float scale,

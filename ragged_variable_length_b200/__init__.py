@@ -37,6 +37,7 @@ RAGGED_MAX_TOKENS = 16384
 RAGGED_PIPELINE_AUTO = 0
 RAGGED_PIPELINE_FUSED = 1
 RAGGED_PIPELINE_SPLIT = 2
+RAGGED_PIPELINE_SYNC = 4
 RAGGED_ATTN_AUTO = 0
 RAGGED_ATTN_STREAMING = 1
 RAGGED_ATTN_RESIDENT = 2
@@ -237,6 +238,35 @@ def ragged_get_device_status(stream=None) -> int:
     return int(val.value)
 
 
+class _PipelineArgs(ctypes.Structure):
+    """The parameters of ragged_pipeline, in order (argument block of _fastcall)."""
+    _fields_ = [("dense_qkv", ctypes.c_void_p), ("keep", ctypes.c_void_p), ("B", ctypes.c_int64),
+                ("L_full", ctypes.c_int64), ("H", ctypes.c_int64), ("head_dim", ctypes.c_int64),
+                ("scale", ctypes.c_float), ("dtype", ctypes.c_int32), ("packed_qkv", ctypes.c_void_p),
+                ("cu_seqlens", ctypes.c_void_p), ("out", ctypes.c_void_p), ("cls_out", ctypes.c_void_p),
+                ("flags", ctypes.c_uint32), ("stream", ctypes.c_void_p)]
+
+
+_fast = None
+
+
+def _fast_forwarder():
+    """The single-crossing forwarder, bound to the loaded library (None if not built)."""
+    global _fast
+    if _fast is None:
+        try:
+            import importlib
+            fc = importlib.import_module(__name__ + "._fastcall")
+        except ImportError:
+            _fast = False
+            return None
+        if fc.args_size() != ctypes.sizeof(_PipelineArgs):
+            raise RuntimeError("_fastcall argument block does not match the binding")
+        fc.bind(ctypes.cast(load().ragged_pipeline, ctypes.c_void_p).value)
+        _fast = fc
+    return _fast or None
+
+
 class Pipeline:
     """Pre-marshalled pack -> attend -> CLS for one (B, L_full, H, dtype) shape.
 
@@ -274,9 +304,23 @@ class Pipeline:
                       c.c_void_p(self.cu_seqlens.data_ptr()), c.c_void_p(self.out.data_ptr()),
                       c.c_void_p(self.cls_out.data_ptr()), c.c_uint32(self.flags), c.c_void_p(_stream(stream)))
         self._fn = load().ragged_pipeline
+        self._block = _PipelineArgs(*[a.value for a in self._args])
+        self._block_sync = _PipelineArgs(*[a.value for a in self._args])
+        self._block_sync.flags = self.flags | RAGGED_PIPELINE_SYNC
+        self._block_addr = ctypes.addressof(self._block)
+        self._block_sync_addr = ctypes.addressof(self._block_sync)
+        self._fc = _fast_forwarder()
 
     def __call__(self) -> None:
-        st = self._fn(*self._args)
+        """Enqueue pack -> attend -> CLS on the bound stream."""
+        st = self._fc.run(self._block_addr) if self._fc else self._fn(*self._args)
+        if st:
+            _check(st)
+
+    def run_sync(self) -> None:
+        """Enqueue the pipeline and return once it has finished (one call)."""
+        st = self._fc.run(self._block_sync_addr) if self._fc else \
+            self._fn(*self._args[:12], ctypes.c_uint32(self.flags | RAGGED_PIPELINE_SYNC), self._args[13])
         if st:
             _check(st)
 

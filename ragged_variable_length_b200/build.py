@@ -51,7 +51,29 @@ def command(out: str, ptxas_verbose: bool = False) -> list:
     return cmd
 
 
+FASTCALL_SRC = os.path.join(CSRC, "fastcall.c")
+
+
+def fastcall_path() -> str:
+    import sysconfig
+    return os.path.join(HERE, "_fastcall" + sysconfig.get_config_var("EXT_SUFFIX"))
+
+
+def build_fastcall(force: bool = False) -> str:
+    """CPython extension that forwards a pre-marshalled ragged_pipeline call."""
+    import sysconfig
+    out = fastcall_path()
+    if not force and os.path.exists(out) and os.path.getmtime(out) >= os.path.getmtime(FASTCALL_SRC):
+        return out
+    tmp = f"{out}.{os.getpid()}.tmp"
+    subprocess.run(["gcc", "-O2", "-Wall", "-shared", "-fPIC", f"-I{sysconfig.get_paths()['include']}",
+                    FASTCALL_SRC, "-o", tmp], check=True)
+    os.replace(tmp, out)
+    return out
+
+
 def build(force: bool = False, ptxas_verbose: bool = False) -> str:
+    build_fastcall(force)
     if not force and not stale():
         return LIB
     tmp = f"{LIB}.{os.getpid()}.tmp"

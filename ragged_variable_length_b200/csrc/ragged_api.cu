@@ -359,9 +359,15 @@ ragged_status ragged_pipeline(const void* dense_qkv, const uint8_t* keep, int64_
     if (H < 1 || H > 65535) return fail(RAGGED_ERR_INVALID_ARG, "H = %lld outside [1, 65535]", (long long)H);
     if (dtype != RAGGED_F16 && dtype != RAGGED_BF16 && dtype != RAGGED_F32)
         return fail(RAGGED_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
-    if ((flags & ~(RAGGED_PIPELINE_FUSED | RAGGED_PIPELINE_SPLIT)) != 0 ||
-        flags == (RAGGED_PIPELINE_FUSED | RAGGED_PIPELINE_SPLIT))
+    if ((flags & ~(RAGGED_PIPELINE_FUSED | RAGGED_PIPELINE_SPLIT | RAGGED_PIPELINE_SYNC)) != 0 ||
+        (flags & (RAGGED_PIPELINE_FUSED | RAGGED_PIPELINE_SPLIT)) == (RAGGED_PIPELINE_FUSED | RAGGED_PIPELINE_SPLIT))
         return fail(RAGGED_ERR_INVALID_ARG, "flags = %u is not a valid pipeline mode", flags);
+    if (flags & RAGGED_PIPELINE_SYNC) {
+        ragged_status st = ragged_pipeline(dense_qkv, keep, B, L_full, H, head_dim, scale, dtype, packed_qkv,
+                                           cu_seqlens, out, cls_out, flags & ~RAGGED_PIPELINE_SYNC, stream);
+        if (st != RAGGED_OK) return st;
+        return cuda_check(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)), "cudaStreamSynchronize");
+    }
     const int64_t esz = dtype == RAGGED_F32 ? 4 : 2;
     const int64_t D = H * head_dim;
     ragged_status st = check_rows(B, L_full, 3 * D * esz);

@@ -143,6 +143,8 @@ def _pipe(lib, **kw):
     (dict(dense=A8), rv.RAGGED_ERR_INVALID_ARG, "16-byte"),
     (dict(out=A8), rv.RAGGED_ERR_INVALID_ARG, "16-byte"),
     (dict(flags=3), rv.RAGGED_ERR_INVALID_ARG, "flags"),
+    (dict(flags=7), rv.RAGGED_ERR_INVALID_ARG, "flags"),
+    (dict(flags=5, dense=A8), rv.RAGGED_ERR_INVALID_ARG, "16-byte"),
     (dict(flags=8), rv.RAGGED_ERR_INVALID_ARG, "flags"),
     (dict(scale=0.0), rv.RAGGED_ERR_INVALID_ARG, "scale"),
     (dict(L=0), rv.RAGGED_ERR_INVALID_ARG, "L_full"),

@@ -121,3 +121,19 @@ def test_empty_batch_fused():
     st = rv.load().ragged_pipeline(None, None, 0, 197, 6, 64, 0.125, 0, None, cu.data_ptr(), None, None,
                                    rv.RAGGED_PIPELINE_FUSED, torch.cuda.current_stream().cuda_stream)
     assert st == rv.RAGGED_OK and cu.item() == 0
+
+
+@pytest.mark.parametrize("flags", [rv.RAGGED_PIPELINE_FUSED, rv.RAGGED_PIPELINE_SPLIT])
+def test_run_sync_matches_enqueue_then_sync(flags):
+    w = synthetic.serving(2, 0.5)
+    p = rv.Pipeline(w.B, w.L_full, w.H, torch.float16, flags=flags)
+    p.dense_qkv.copy_(to_device(w.qkv, "f16"))
+    p.keep.copy_(torch.from_numpy(w.keep))
+    p()
+    torch.cuda.synchronize()
+    cls_ref = p.cls_out.clone()
+    p.cls_out.zero_()
+    p.run_sync()                      # returns with the results in place
+    assert torch.equal(p.cls_out, cls_ref)
+    packed_o, cu_o = oracle.pack(w.qkv, w.keep)
+    assert np.array_equal(p.cu_seqlens.cpu().numpy(), cu_o)
