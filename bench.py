@@ -41,6 +41,51 @@ L2_BYTES = 126 * 1024 * 1024
 CASES = [(B, p) for B in synthetic.SERVING_BATCHES for p in synthetic.SERVING_RATES]
 
 
+def max_over_ranks(value: float, dist, device=None) -> float:
+    """The largest of every rank's value (the job's time is its slowest rank's)."""
+    if not dist:
+        return float(value)
+    import torch
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def us_per_call(ms: float, steps: int, calls_per_step: int, world: int) -> float:
+    """Microseconds per call over all calls of all ranks, from the max-over-ranks time."""
+    return ms * 1000.0 / (steps * calls_per_step * world)
+
+
+FUSED_SOURCES = ("attn_resident.cuh", "pack.cuh", "mma_common.cuh", "common.cuh")
+TRAFFIC_RECORD = os.path.join(ROOT, "profiles", "fused_serving_traffic.txt")
+
+
+def fused_source_hash() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for name in FUSED_SOURCES:
+        with open(os.path.join(ROOT, "ragged_variable_length_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def recorded_traffic():
+    """DRAM bytes per fused launch from the committed ncu record, or None when the
+    kernel sources changed since the counters were taken."""
+    try:
+        fields = {}
+        with open(TRAFFIC_RECORD) as f:
+            for line in f:
+                if ":" in line and not line.startswith("#"):
+                    k, v = line.split(":", 1)
+                    fields[k.strip()] = v.strip()
+        if fields.get("kernel_source_sha256") != fused_source_hash():
+            return None
+        return int(fields["dram_bytes_per_launch_mean"])
+    except (OSError, KeyError, ValueError):
+        return None
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -210,13 +255,9 @@ def run_ours(args, rank, world, dist):
     if dist:
         dist.barrier()
     clocks = sampler.stop()
-    ms = e0.elapsed_time(e1)
-    if dist:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(e0.elapsed_time(e1), dist, dev)
     calls = args.steps * len(CASES) * world
-    us_per_call = ms * 1000.0 / calls
+    value_us = us_per_call(ms, args.steps, len(CASES), world)
 
     # The same calls without the graph: one C call per pipeline run.
     if dist:
@@ -228,12 +269,8 @@ def run_ours(args, rank, world, dist):
         step_direct(s)
     d1.record(stream)
     torch.cuda.synchronize()
-    direct_ms = d0.elapsed_time(d1)
-    if dist:
-        t = torch.tensor([direct_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        direct_ms = float(t.item())
-    direct_us = direct_ms * 1000.0 / calls
+    direct_ms = max_over_ranks(d0.elapsed_time(d1), dist, dev)
+    direct_us = us_per_call(direct_ms, args.steps, len(CASES), world)
 
     # ---- per-call host / device / total split, per case ----
     detail = {}
@@ -294,12 +331,8 @@ def run_ours(args, rank, world, dist):
         e2e_step(s)
     x1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = x0.elapsed_time(x1)
-    if dist:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_us = e2e_ms * 1000.0 / calls
+    e2e_ms = max_over_ranks(x0.elapsed_time(x1), dist, dev)
+    e2e_us = us_per_call(e2e_ms, args.steps, len(CASES), world)
     # the last step's CLS rows must match the device result
     ok_e2e = all(torch.equal(host_in[((args.steps - 1) % ncopies, i)][2], pl.cls_out.cpu())
                  for i, pl in enumerate(pipes[(args.steps - 1) % ncopies]))
@@ -365,7 +398,7 @@ def run_ours(args, rank, world, dist):
     b_pack = float(np.mean([pack_bytes(w_) for _, w_ in all_pw]))
     flops = float(np.mean([w_.useful_flops() for _, w_ in all_pw]))
     roofline = {"bound": "hbm", "achieved": round(b_fused / t_fused / 1e9, 2), "peak": hbm_peak,
-                "unit": "GB/s", "frac": round(b_fused / t_fused / 1e9 / hbm_peak, 4), "traffic": None,
+                "unit": "GB/s", "frac": round(b_fused / t_fused / 1e9 / hbm_peak, 4), "traffic": recorded_traffic(),
                 "kernel": "attn_resident_kernel<__half, DenseRows> (fused pack + attention + CLS)",
                 "avg_launch_us": round(t_fused * 1e6, 3), "bytes_per_launch": int(b_fused),
                 "launches_timed": 3 * len(all_pw), "peak_kind": peak_kind,
@@ -378,7 +411,7 @@ def run_ours(args, rank, world, dist):
 
     # ---- larger workloads: attention roofline (single GPU, same kernel family) ----
     larger = {}
-    if not args.quick:
+    if not args.quick and world == 1:
         for name, make, copies in (("deit_b_p80_b32", lambda c: synthetic.make_workload(
                                         "deit_b_p80_b32", 32, 197, 12,
                                         synthetic.deit_b_pruned80().lengths, "bf16", 1002, 1 + c), 36),
@@ -426,7 +459,7 @@ def run_ours(args, rank, world, dist):
 
     gpu_launches = 1 * args.steps * len(CASES)   # one fused launch per call
     hw = {"metric": "ragged attn µs/call (host+device) at BS1-4; useful TFLOP/s & % roofline",
-          "value": round(us_per_call, 3), "unit": "µs/call", "n_gpus": world, "steps": args.steps,
+          "value": round(value_us, 3), "unit": "µs/call", "n_gpus": world, "steps": args.steps,
           "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 4), "higher_is_better": False,
           "scaling": "weak", "vs_baseline": None, "dtype": "f16", "data": "synthetic",
           "config": {"workload": "serving_deit_s_b1-4_p0-80", "B": list(synthetic.SERVING_BATCHES),
@@ -539,6 +572,43 @@ def run_reference(args, rank, world):
     }), flush=True)
 
 
+PROFILE_CASES = ("serving", "hires")
+
+
+def run_profile_case(case: str) -> None:
+    """One untimed pass of a workload, for an ncu capture of its kernels.
+
+    serving: the fused pipeline once on each of the 12 serving batches.
+    hires:   the 384x384 B=64 workload packed, then attention twice with the
+             streaming mma.sync kernel and twice with the tcgen05 kernel.
+    """
+    import torch
+    import ragged_variable_length_b200 as rv
+    torch.cuda.set_device(0)
+    if case == "serving":
+        pls = []
+        for B, p in CASES:
+            w = synthetic.serving(B, p)
+            pl = rv.Pipeline(w.B, w.L_full, w.H, torch.float16, flags=rv.RAGGED_PIPELINE_FUSED)
+            pl.dense_qkv.copy_(torch.from_numpy(w.qkv))
+            pl.keep.copy_(torch.from_numpy(w.keep))
+            pls.append(pl)
+        torch.cuda.synchronize()
+        for pl in pls:
+            pl()
+    elif case == "hires":
+        w = synthetic.hires_384()
+        pl = rv.Pipeline(w.B, w.L_full, w.H, torch.bfloat16, flags=rv.RAGGED_PIPELINE_SPLIT)
+        pl.dense_qkv.view(torch.int16).copy_(torch.from_numpy(w.qkv.view(np.int16)))
+        pl.keep.copy_(torch.from_numpy(w.keep))
+        for kern in (rv.RAGGED_ATTN_STREAMING, rv.RAGGED_ATTN_TCGEN05):
+            rv.ragged_set_attn_kernel(kern)
+            pl()
+            pl()
+        rv.ragged_set_attn_kernel(rv.RAGGED_ATTN_AUTO)
+    torch.cuda.synchronize()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -546,7 +616,11 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--quick", action="store_true", help="skip the larger workloads and the CPU baseline")
+    ap.add_argument("--profile", choices=PROFILE_CASES, help="one untimed pass of a workload (for ncu), no JSON")
     args = ap.parse_args()
+    if args.profile:
+        run_profile_case(args.profile)
+        return
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -401,26 +401,73 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ---------------------------------------------------------------------------
 // Streaming variant: two CTAs per SM.
 //
-// Same operation and roles as attn_tc05_kernel, but the K/V tiles of a
-// sequence flow through a 3-stage shared-memory ring (loads run two tiles
-// ahead) and TMEM holds only two 64-column S buffers and O (256 columns), so
-// two CTAs share each SM and one's softmax overlaps the other's loads and
-// MMAs.  Within a CTA, S = Q K^T of tile t + 1 is issued before the softmax of
-// tile t.  The softmax is single-pass: each row keeps a reference maximum and
-// rescales its running sum and O (in TMEM) only when a tile raises the row
-// maximum by more than 2^8 in base 2; otherwise the probabilities
-// exp2(s - reference) stay below 256 and the reference is kept.  The final
-// division by the running sum makes the result independent of the reference.
+// Same operation as attn_tc05_kernel, but the K/V tiles of a sequence flow
+// through a 5-stage shared-memory ring (loads run four tiles ahead), and the
+// probabilities never touch shared memory: each softmax thread stores its
+// row of P into TMEM (16-bit values packed two per column, row = lane) and
+// the P V product reads its A operand from TMEM.  TMEM per CTA (256 columns):
+//   [0, 64) and [64, 128)   S of tiles t (even / odd)
+//   [128, 192)              P: two f16 slots of 32 columns, or the bf16 hi/lo pair
+//   [192, 256)              O
+// so two CTAs share each SM.  S = Q K^T of tile t + 1 is issued before the
+// softmax of tile t.  The softmax is single-pass: each row keeps a reference
+// maximum and rescales its running sum and O (in TMEM) only when a tile
+// raises the row maximum by more than 2^8 in base 2; otherwise the
+// probabilities exp2(s - reference) stay below 256 and the reference is kept.
+// The final division by the running sum makes the result independent of the
+// reference.  Warps whose 32 query rows all lie past the sequence end skip
+// the softmax; fully-masked 16-key groups of the last tile are skipped too.
 // ---------------------------------------------------------------------------
 
 constexpr uint32_t kStreamTmemCols = 256;
-constexpr uint32_t kStreamOCol = 128;          // S buffers at columns 0 and 64
-constexpr int kStages = 3;
+constexpr uint32_t kStreamPCol = 128;
+constexpr uint32_t kStreamOCol = 192;
+constexpr int kStages = 5;
 constexpr float kRescaleThreshold = 8.f;       // log2 units
 
-__host__ __device__ constexpr int stream_smem_bytes(int p_parts) {
-    // alignment slack, Q, K/V ring, P (two slots for f16, one hi/lo pair for bf16)
-    return 1024 + kQBytes + kStages * 2 * kKVTileBytes + 2 * kPTileBytes;
+__host__ __device__ constexpr int stream_smem_bytes(int /*p_parts*/) {
+    return 1024 + kQBytes + kStages * 2 * kKVTileBytes;   // alignment slack, Q, K/V ring
+}
+
+// 32 consecutive 32-bit TMEM columns of this thread's lane <- v.
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};\n"
+        :
+        : "r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+          "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]),
+          "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]),
+          "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+        : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// 64 consecutive fp32 columns of this thread's TMEM lane, one load and one wait.
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&v)[64]) {
+    uint32_t r[64];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x64.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%64];\n\t"
+        "tcgen05.wait::ld.sync.aligned;\n"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]), "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
+        : "r"(taddr)
+        : "memory");
+#pragma unroll
+    for (int i = 0; i < 64; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+
+
+// O (TMEM) += P (TMEM, A operand) x V (shared memory, B operand).
+__device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                           uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, {%5, %6, %7, %8}, p;\n\t}\n"
+        :
+        : "r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(0), "r"(0), "r"(0), "r"(0)
+        : "memory");
 }
 
 template <typename T>
@@ -428,7 +475,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     attn_tc05_stream_kernel(PackedRows src, float scale_log2, int H, uint16_t* __restrict__ out,
                             int64_t out_tok_stride, uint16_t* __restrict__ cls_out) {
     extern __shared__ uint8_t smem_raw[];
-    // mbarriers: 0, 1: S buffer ready; 2, 3: P V product of slot done
+    // mbarriers: 0, 1: S buffer ready; 2, 3: P V product of tile parity done
     __shared__ __align__(8) uint64_t s_mbar[4];
     __shared__ uint32_t s_tmem;
     __shared__ int s_fail;
@@ -439,15 +486,12 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int q0 = qt * kRows;
     if (q0 >= len) return;
     const int nt = (len + kTileN - 1) / kTileN;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int tid = threadIdx.x, warp = tid >> 5;
     constexpr int kParts = Cvt<T>::kParts;
-    constexpr int kSlots = 2 / kParts;     // f16: two P slots; bf16: one hi/lo pair
 
     const uint32_t raw = smem_addr(smem_raw);
     const uint32_t sQ = (raw + 1023u) & ~1023u;
     const uint32_t sRing = sQ + kQBytes;                         // stage s: K at +s*16K, V at +8K
-    const uint32_t sP = sRing + kStages * 2 * kKVTileBytes;
-    uint8_t* gP = smem_raw + (sP - raw);
     auto stage_k = [&](int t) { return sRing + (t % kStages) * 2 * kKVTileBytes; };
     auto stage_v = [&](int t) { return stage_k(t) + kKVTileBytes; };
     auto load_kv = [&](int t) {
@@ -456,10 +500,11 @@ __global__ void __launch_bounds__(kThreads, 2)
         cp_async_commit();
     };
 
-    // Loads: group 0 = Q + tile 0, then one group per tile, two tiles ahead.
+    // Loads: group 0 = Q + tile 0, then one group per tile, up to 4 ahead.
     resident::load_tile<kRows>(sQ, src, 0, q0, len);
     load_kv(0);
-    if (nt > 1) load_kv(1);
+    for (int t = 1; t < min(nt, kStages - 1); ++t) load_kv(t);
+    int issued = min(nt, kStages - 1);    // tiles whose loads are in flight or done
 
     const uint32_t mbar0 = smem_addr(&s_mbar[0]);
     if (tid == 0) {
@@ -482,12 +527,12 @@ __global__ void __launch_bounds__(kThreads, 2)
     const uint32_t idesc_qk = make_idesc(Cvt<T>::kFormat, 0, kTileN);
     const uint32_t idesc_pv = make_idesc(Cvt<T>::kFormat, 1, 64);
     const int row = q0 + tid;
+    const bool warp_rows = q0 + warp * 32 < len;   // this warp owns at least one real row
 
-    // Waits until this thread's copies of tile t have landed, leaving
-    // `pending` later groups in flight, and publishes them to the tensor core;
-    // includes the CTA barrier.
-    auto tile_landed = [&](int pending) {
-        if (pending) cp_async_wait<1>(); else cp_async_wait<0>();
+    // Waits until tile t's copies have landed (leaving the tiles issued after
+    // it in flight), publishes them to the tensor core; includes the barrier.
+    auto tile_landed = [&](int t) {
+        resident::cp_async_wait_pending(issued - 1 - t);
         fence_async_smem();
         fence_before_sync();
         __syncthreads();
@@ -506,123 +551,132 @@ __global__ void __launch_bounds__(kThreads, 2)
         if (!mbar_wait(mbar, static_cast<uint32_t>((t >> 1) & 1))) atomicExch(&s_fail, 1);
     };
 
-    tile_landed(nt > 1 ? 1 : 0);
+    tile_landed(0);
     if (tid == 0) issue_qk(0);
+
+    // Products confirmed finished, per thread (every thread confirms the same
+    // tiles, so the value is uniform where the refill decision reads it).  A
+    // product's mbarrier is waited on only while the next product on the same
+    // barrier has not been issued, so a parity wait never misses a phase.
+    int pv_seen = -1;
+    auto confirm_pv = [&](int x) {
+        if (x > pv_seen) {
+            wait_tile_event(mbar0 + 16 + 8 * (x & 1), x);
+            pv_seen = x;
+        }
+    };
+    // f16 keeps two P slots (slot t & 1), bf16 one hi/lo pair: writing P of tile
+    // t needs the product of tile t - 2 (f16) or t - 1 (bf16) finished.
+    constexpr int kPLag = kParts == 2 ? 1 : 2;
 
     float m_ref = -INFINITY;   // reference maximum (log2 units) of this row
     float l = 0.f;
     for (int t = 0; t < nt; ++t) {
-        // (a) S of tile t + 1 (landed: issued one iteration ago) is computed
-        // while this tile's softmax runs; its S buffer was last read by the
-        // softmax of tile t - 1, which is finished.
+        // (a) S of tile t + 1 is computed while this tile's softmax runs; its
+        // S buffer was last read by the softmax of tile t - 1, which is done.
         if (t + 1 < nt) {
-            tile_landed(0);
+            tile_landed(t + 1);
             if (s_fail) break;
             if (tid == 0) issue_qk(t + 1);
         }
-        // (b) Once the product of tile t - 1 is done (and with it every earlier
-        // product, so both P slots and the stage of tile t - 1 are free),
-        // refill that stage with tile t + 2.
-        if (t >= 1) wait_tile_event(mbar0 + 16 + 8 * ((t - 1) & 1), t - 1);
-        if (t + 2 < nt) load_kv(t + 2);
-        // (c) S of tile t.
+        // (b) S of tile t.
         wait_tile_event(mbar0 + 8 * (t & 1), t);
         fence_after_sync();
 
-        float sv[4][16];
-        float mt = -INFINITY;
+        const int valid = min(kTileN, len - t * kTileN);   // keys of this tile
+        if (warp_rows) {
+            float sv[64];
+            tmem_ld64(t_lane + static_cast<uint32_t>((t & 1) * kTileN), sv);
+            if (valid < kTileN) {
 #pragma unroll
-        for (int g = 0; g < 4; ++g) {
-            tmem_ld16(t_lane + static_cast<uint32_t>((t & 1) * kTileN + g * 16), sv[g]);
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const bool ok = t * kTileN + g * 16 + i < len;
-                sv[g][i] = ok ? sv[g][i] * scale_log2 : -INFINITY;
-                mt = fmaxf(mt, sv[g][i]);
+                for (int i = 0; i < 64; ++i)
+                    if (i >= valid) sv[i] = -INFINITY;
             }
-        }
-        // (d) Rescale only when the tile's maximum exceeds the reference by
-        // more than the threshold (always for the first tile).
-        const bool grow = mt > m_ref + kRescaleThreshold;
-        float alpha = 1.f;
-        if (grow) {
-            alpha = fast_exp2_guard(m_ref - mt);
-            l *= alpha;
-            m_ref = mt;
-        }
-        if (t > 0 && __any_sync(0xffffffffu, grow)) {
-            // O holds the (finished, see (b)) products of tiles 0 .. t - 1:
-            // scale this warp's rows in TMEM; rows that keep their reference
-            // are multiplied by 1.
+            float mx = -INFINITY;
 #pragma unroll
-            for (int g = 0; g < 4; ++g) {
-                float ov[16];
-                tmem_ld16(t_lane + kStreamOCol + g * 16, ov);
-#pragma unroll
-                for (int i = 0; i < 16; ++i) ov[i] *= alpha;
-                tmem_st16(t_lane + kStreamOCol + g * 16, ov);
+            for (int i = 0; i < 64; ++i) mx = fmaxf(mx, sv[i]);
+            // (c) Rescale only when the tile's maximum exceeds the reference by
+            // more than the threshold (always for the first tile).
+            const float mt = mx * scale_log2;
+            const bool grow = mt > m_ref + kRescaleThreshold;
+            float alpha = 1.f;
+            if (grow) {
+                alpha = fast_exp2_guard(m_ref - mt);
+                l *= alpha;
+                m_ref = mt;
             }
-        }
-
-        uint8_t* p_base = gP + (kSlots == 2 ? (t & 1) : 0) * kPTileBytes;
+            if (t > 0 && __any_sync(0xffffffffu, grow)) {
+                // O must hold the finished products of tiles 0 .. t - 1.
+                confirm_pv(t - 1);
+                fence_after_sync();
+                float ov[64];
+                tmem_ld64(t_lane + kStreamOCol, ov);
 #pragma unroll
-        for (int g = 0; g < 4; ++g) {
+                for (int g = 0; g < 4; ++g) {
+                    float part[16];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                sv[g][i] = mma_attn::fast_exp2(sv[g][i] - m_ref);   // -inf -> 0
-                l += sv[g][i];
-            }
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                uint32_t w[4];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) w[i] = Cvt<T>::pack(sv[g][half * 8 + 2 * i], sv[g][half * 8 + 2 * i + 1]);
-                const int chunk = g * 2 + half;
-                *reinterpret_cast<uint4*>(p_base + swz(tid, chunk)) = make_uint4(w[0], w[1], w[2], w[3]);
-                if constexpr (kParts == 2) {
-                    uint32_t r[4];
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        __nv_bfloat162 hb = *reinterpret_cast<__nv_bfloat162*>(&w[i]);
-                        const float2 f = __bfloat1622float2(hb);
-                        r[i] = Cvt<T>::pack(sv[g][half * 8 + 2 * i] - f.x, sv[g][half * 8 + 2 * i + 1] - f.y);
-                    }
-                    *reinterpret_cast<uint4*>(p_base + kPTileBytes + swz(tid, chunk)) =
-                        make_uint4(r[0], r[1], r[2], r[3]);
+                    for (int i = 0; i < 16; ++i) part[i] = ov[g * 16 + i] * alpha;
+                    tmem_st16(t_lane + kStreamOCol + g * 16, part);
                 }
             }
+            // (d) P = exp2(s * scale - reference) (masked keys -> 0).
+            uint32_t p_hi[32], p_lo[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                const float a = mma_attn::fast_exp2(fmaf(sv[2 * i], scale_log2, -m_ref));   // -inf -> 0
+                const float c = mma_attn::fast_exp2(fmaf(sv[2 * i + 1], scale_log2, -m_ref));
+                l += a + c;
+                const uint32_t w = Cvt<T>::pack(a, c);
+                p_hi[i] = w;
+                if constexpr (kParts == 2) {
+                    __nv_bfloat162 hb = *reinterpret_cast<const __nv_bfloat162*>(&w);
+                    const float2 f = __bfloat1622float2(hb);
+                    p_lo[i] = Cvt<T>::pack(a - f.x, c - f.y);
+                }
+            }
+            // (e) The P slot must be free before it is overwritten.
+            if (t >= kPLag) confirm_pv(t - kPLag);
+            fence_after_sync();
+            const uint32_t p_col = t_lane + kStreamPCol + (kParts == 2 ? 0u : static_cast<uint32_t>((t & 1) * 32));
+            tmem_st32(p_col, p_hi);
+            if constexpr (kParts == 2) tmem_st32(p_col + 32, p_lo);
+            tmem_wait_st();
+        } else if (t >= kPLag) {
+            confirm_pv(t - kPLag);
         }
-        fence_async_smem();
+        // (f) Refill: the stage of tile x is free once Q K^T(x) and P V(x) are
+        // done, which holds for x <= t - kPLag (confirmed above).
+        if (issued < nt && issued - kStages <= t - kPLag) {
+            load_kv(issued);
+            ++issued;
+        }
         fence_before_sync();
         __syncthreads();
         if (s_fail) break;
         if (tid == 0) {
             fence_after_sync();
-            const uint32_t p_addr = sP + (kSlots == 2 ? (t & 1) : 0) * kPTileBytes;
+            const uint32_t p_addr = tmem + kStreamPCol + (kParts == 2 ? 0u : static_cast<uint32_t>((t & 1) * 32));
 #pragma unroll
             for (int part = 0; part < kParts; ++part)
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
-                    mma_f16(tmem + kStreamOCol, make_sdesc(p_addr + part * kPTileBytes + ks * 32),
-                            make_sdesc(stage_v(t) + ks * 2048), idesc_pv, (t > 0 || part > 0 || ks > 0) ? 1u : 0u);
+                    mma_f16_ts(tmem + kStreamOCol, p_addr + part * 32 + ks * 8, make_sdesc(stage_v(t) + ks * 2048),
+                               idesc_pv, (t > 0 || part > 0 || ks > 0) ? 1u : 0u);
             mma_commit(mbar0 + 16 + 8 * (t & 1));
         }
     }
 
     // Epilogue: wait for the last product, O / l.
     if (!s_fail) {
-        wait_tile_event(mbar0 + 16 + 8 * ((nt - 1) & 1), nt - 1);
-        if (!s_fail) {
+        confirm_pv(nt - 1);
+        if (!s_fail && warp_rows) {
             fence_after_sync();
             const float inv = 1.f / l;
+            float v[64];
+            tmem_ld64(t_lane + kStreamOCol, v);
             uint32_t w[32];
 #pragma unroll
-            for (int g = 0; g < 4; ++g) {
-                float v[16];
-                tmem_ld16(t_lane + kStreamOCol + g * 16, v);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) w[g * 8 + i] = Cvt<T>::pack(v[2 * i] * inv, v[2 * i + 1] * inv);
-            }
+            for (int i = 0; i < 32; ++i) w[i] = Cvt<T>::pack(v[2 * i] * inv, v[2 * i + 1] * inv);
             if (row < len) {
                 uint4* dst = reinterpret_cast<uint4*>(out + static_cast<int64_t>(start + row) * out_tok_stride +
                                                       h * 64);
@@ -646,7 +700,6 @@ __global__ void __launch_bounds__(kThreads, 2)
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kStreamTmemCols)
                      : "memory");
     }
-    (void)lane;
 }
 
 }  // namespace tc05

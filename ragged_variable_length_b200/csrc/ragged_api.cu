@@ -308,11 +308,14 @@ ragged_status ragged_attn_fwd(const void* q, const void* k, const void* v, int64
     // single-tile sequences; other launches stream K/V tiles.
     const int res_tiles = static_cast<int>((max_seqlen + 63) / 64);
     int kernel_choice = g_attn_kernel.load(std::memory_order_relaxed);
-    if (kernel_choice == RAGGED_ATTN_AUTO)
-        kernel_choice = (max_seqlen <= ragged::resident::kMaxKeys &&
-                         (res_tiles == 1 || resident_ksplit(B, H, res_tiles) > 1))
-                            ? RAGGED_ATTN_RESIDENT
-                            : RAGGED_ATTN_STREAMING;
+    if (kernel_choice == RAGGED_ATTN_AUTO) {
+        if (max_seqlen <= ragged::resident::kMaxKeys && (res_tiles == 1 || resident_ksplit(B, H, res_tiles) > 1))
+            kernel_choice = RAGGED_ATTN_RESIDENT;
+        else if (res_tiles > 4)
+            kernel_choice = RAGGED_ATTN_TCGEN05;   // long sequences: many key tiles per query tile
+        else
+            kernel_choice = RAGGED_ATTN_STREAMING;
+    }
     if (kernel_choice == RAGGED_ATTN_RESIDENT && max_seqlen > ragged::resident::kMaxKeys)
         return fail(RAGGED_ERR_UNSUPPORTED, "the resident attention kernel holds at most 640 keys");
     ragged::resident::PackedRows src{static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(k),

@@ -98,10 +98,12 @@ def test_streaming_kernel_under_a_loose_bound(dtype):
 
 
 @pytest.mark.parametrize("dtype", ["f16", "bf16"])
-def test_long_sequences_streaming_kernel(dtype):
-    """L_full above the resident limit (640 keys) runs the streaming kernel."""
+@pytest.mark.parametrize("kernel", ["auto", "streaming"])
+def test_long_sequences_above_the_resident_limit(dtype, kernel):
+    """L_full above the resident limit (640 keys): the streaming kernel, and
+    AUTO (which picks tcgen05 for sequences over 256 keys)."""
     w = synthetic.make_workload("long", 4, 1000, 2, [1000, 700, 641, 65], dtype, 81)
-    check_against_oracle(w)
+    check_against_oracle(w, kernel=kernel)
 
 
 def test_kernel_limits_are_reported():
