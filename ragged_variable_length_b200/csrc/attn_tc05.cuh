@@ -470,13 +470,31 @@ __device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uin
         : "memory");
 }
 
+// Warp roles: warps 0-3 (128 threads, one per query row) load K/V tiles with
+// cp.async and run the softmax; warp 4 issues every tcgen05.mma.  They hand
+// off through mbarriers only, so no CTA-wide barrier sits in the tile loop:
+//   kv_ready[stage]  (128 arrivals) the tile in that ring stage has landed and
+//                    is visible to the tensor core;
+//   s_ready[t & 1]   (commit)       S of tile t is in TMEM;
+//   p_ready[t & 1]   (128 arrivals) P of tile t is in TMEM and S of tile t has
+//                    been read, so that S buffer may be overwritten;
+//   pv_done[t & 1]   (commit)       the P V product of tile t (and everything
+//                    issued before it) has finished.
+// The MMA warp issues Q K^T(t) as soon as tile t has landed, then P V(t - 1)
+// once P(t - 1) is ready, so the S of the next tile is always computed while
+// the softmax of the current one runs.
+constexpr int kStreamThreads = 160;
+constexpr int kSoftmaxThreads = 128;
+
 template <typename T>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kStreamThreads, 2)
     attn_tc05_stream_kernel(PackedRows src, float scale_log2, int H, uint16_t* __restrict__ out,
                             int64_t out_tok_stride, uint16_t* __restrict__ cls_out) {
     extern __shared__ uint8_t smem_raw[];
-    // mbarriers: 0, 1: S buffer ready; 2, 3: P V product of tile parity done
-    __shared__ __align__(8) uint64_t s_mbar[4];
+    __shared__ __align__(8) uint64_t s_kv_ready[kStages];
+    __shared__ __align__(8) uint64_t s_s_ready[2];
+    __shared__ __align__(8) uint64_t s_p_ready[2];
+    __shared__ __align__(8) uint64_t s_pv_done[2];
     __shared__ uint32_t s_tmem;
     __shared__ int s_fail;
 
@@ -487,6 +505,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     if (q0 >= len) return;
     const int nt = (len + kTileN - 1) / kTileN;
     const int tid = threadIdx.x, warp = tid >> 5;
+    const bool mma_warp = warp == 4;
     constexpr int kParts = Cvt<T>::kParts;
 
     const uint32_t raw = smem_addr(smem_raw);
@@ -500,15 +519,25 @@ __global__ void __launch_bounds__(kThreads, 2)
         cp_async_commit();
     };
 
-    // Loads: group 0 = Q + tile 0, then one group per tile, up to 4 ahead.
-    resident::load_tile<kRows>(sQ, src, 0, q0, len);
-    load_kv(0);
-    for (int t = 1; t < min(nt, kStages - 1); ++t) load_kv(t);
-    int issued = min(nt, kStages - 1);    // tiles whose loads are in flight or done
+    // Loads by the softmax threads: group 0 = Q + tile 0, then one group per
+    // tile, up to four ahead.
+    int issued = min(nt, kStages - 1);
+    if (!mma_warp) {
+        resident::load_tile<kRows>(sQ, src, 0, q0, len);
+        for (int t = 0; t < issued; ++t) load_kv(t);
+    }
 
-    const uint32_t mbar0 = smem_addr(&s_mbar[0]);
+    const uint32_t kv_ready0 = smem_addr(&s_kv_ready[0]);
+    const uint32_t s_ready0 = smem_addr(&s_s_ready[0]);
+    const uint32_t p_ready0 = smem_addr(&s_p_ready[0]);
+    const uint32_t pv_done0 = smem_addr(&s_pv_done[0]);
     if (tid == 0) {
-        for (int i = 0; i < 4; ++i) mbar_init(mbar0 + 8 * i, 1);
+        for (int i = 0; i < kStages; ++i) mbar_init(kv_ready0 + 8 * i, kSoftmaxThreads);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(s_ready0 + 8 * i, 1);
+            mbar_init(p_ready0 + 8 * i, kSoftmaxThreads);
+            mbar_init(pv_done0 + 8 * i, 1);
+        }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         s_fail = 0;
     }
@@ -522,176 +551,174 @@ __global__ void __launch_bounds__(kThreads, 2)
     __syncthreads();
     fence_after_sync();
     const uint32_t tmem = s_tmem;
-    const uint32_t t_lane = tmem + (static_cast<uint32_t>(warp * 32) << 16);
 
-    const uint32_t idesc_qk = make_idesc(Cvt<T>::kFormat, 0, kTileN);
-    const uint32_t idesc_pv = make_idesc(Cvt<T>::kFormat, 1, 64);
-    const int row = q0 + tid;
-    const bool warp_rows = q0 + warp * 32 < len;   // this warp owns at least one real row
-
-    // Waits until tile t's copies have landed (leaving the tiles issued after
-    // it in flight), publishes them to the tensor core; includes the barrier.
-    auto tile_landed = [&](int t) {
-        resident::cp_async_wait_pending(issued - 1 - t);
-        fence_async_smem();
-        fence_before_sync();
-        __syncthreads();
+    // Event waits; an event is awaited only while the next event on the same
+    // barrier cannot have completed yet, so a parity wait never misses a phase.
+    auto wait_event = [&](uint32_t mbar, uint32_t parity) {
+        if (!mbar_wait(mbar, parity)) atomicExch(&s_fail, 1);
     };
-    auto issue_qk = [&](int t) {   // by thread 0, after tile t has landed
-        fence_after_sync();
-        const uint32_t d = tmem + static_cast<uint32_t>((t & 1) * kTileN);
-#pragma unroll
-        for (int ks = 0; ks < 4; ++ks)
-            mma_f16(d, make_sdesc(sQ + ks * 32), make_sdesc(stage_k(t) + ks * 32), idesc_qk, ks > 0);
-        mma_commit(mbar0 + 8 * (t & 1));
-    };
-    // mbarrier k (k = 0, 1) completes once per tile t with t % 2 == k, so the
-    // wait for tile t uses parity (t / 2) & 1.
-    auto wait_tile_event = [&](uint32_t mbar, int t) {
-        if (!mbar_wait(mbar, static_cast<uint32_t>((t >> 1) & 1))) atomicExch(&s_fail, 1);
+    auto arrive = [&](uint32_t mbar) {
+        asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(mbar) : "memory");
     };
 
-    tile_landed(0);
-    if (tid == 0) issue_qk(0);
-
-    // Products confirmed finished, per thread (every thread confirms the same
-    // tiles, so the value is uniform where the refill decision reads it).  A
-    // product's mbarrier is waited on only while the next product on the same
-    // barrier has not been issued, so a parity wait never misses a phase.
-    int pv_seen = -1;
-    auto confirm_pv = [&](int x) {
-        if (x > pv_seen) {
-            wait_tile_event(mbar0 + 16 + 8 * (x & 1), x);
-            pv_seen = x;
-        }
-    };
-    // f16 keeps two P slots (slot t & 1), bf16 one hi/lo pair: writing P of tile
-    // t needs the product of tile t - 2 (f16) or t - 1 (bf16) finished.
-    constexpr int kPLag = kParts == 2 ? 1 : 2;
-
-    float m_ref = -INFINITY;   // reference maximum (log2 units) of this row
-    float l = 0.f;
-    for (int t = 0; t < nt; ++t) {
-        // (a) S of tile t + 1 is computed while this tile's softmax runs; its
-        // S buffer was last read by the softmax of tile t - 1, which is done.
-        if (t + 1 < nt) {
-            tile_landed(t + 1);
-            if (s_fail) break;
-            if (tid == 0) issue_qk(t + 1);
-        }
-        // (b) S of tile t.
-        wait_tile_event(mbar0 + 8 * (t & 1), t);
-        fence_after_sync();
-
-        const int valid = min(kTileN, len - t * kTileN);   // keys of this tile
-        if (warp_rows) {
-            float sv[64];
-            tmem_ld64(t_lane + static_cast<uint32_t>((t & 1) * kTileN), sv);
-            if (valid < kTileN) {
-#pragma unroll
-                for (int i = 0; i < 64; ++i)
-                    if (i >= valid) sv[i] = -INFINITY;
-            }
-            float mx = -INFINITY;
-#pragma unroll
-            for (int i = 0; i < 64; ++i) mx = fmaxf(mx, sv[i]);
-            // (c) Rescale only when the tile's maximum exceeds the reference by
-            // more than the threshold (always for the first tile).
-            const float mt = mx * scale_log2;
-            const bool grow = mt > m_ref + kRescaleThreshold;
-            float alpha = 1.f;
-            if (grow) {
-                alpha = fast_exp2_guard(m_ref - mt);
-                l *= alpha;
-                m_ref = mt;
-            }
-            if (t > 0 && __any_sync(0xffffffffu, grow)) {
-                // O must hold the finished products of tiles 0 .. t - 1.
-                confirm_pv(t - 1);
+    if (mma_warp) {
+        // ---------------- MMA issuer (one thread) ----------------
+        if ((tid & 31) == 0) {
+            const uint32_t idesc_qk = make_idesc(Cvt<T>::kFormat, 0, kTileN);
+            const uint32_t idesc_pv = make_idesc(Cvt<T>::kFormat, 1, 64);
+            auto issue_pv = [&](int t) {   // P V of tile t, once P(t) is ready
+                wait_event(p_ready0 + 8 * (t & 1), (t >> 1) & 1);
                 fence_after_sync();
-                float ov[64];
-                tmem_ld64(t_lane + kStreamOCol, ov);
+                const uint32_t p_addr = tmem + kStreamPCol + (kParts == 2 ? 0u : static_cast<uint32_t>((t & 1) * 32));
 #pragma unroll
-                for (int g = 0; g < 4; ++g) {
-                    float part[16];
+                for (int part = 0; part < kParts; ++part)
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) part[i] = ov[g * 16 + i] * alpha;
-                    tmem_st16(t_lane + kStreamOCol + g * 16, part);
-                }
-            }
-            // (d) P = exp2(s * scale - reference) (masked keys -> 0).
-            uint32_t p_hi[32], p_lo[32];
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                const float a = mma_attn::fast_exp2(fmaf(sv[2 * i], scale_log2, -m_ref));   // -inf -> 0
-                const float c = mma_attn::fast_exp2(fmaf(sv[2 * i + 1], scale_log2, -m_ref));
-                l += a + c;
-                const uint32_t w = Cvt<T>::pack(a, c);
-                p_hi[i] = w;
-                if constexpr (kParts == 2) {
-                    __nv_bfloat162 hb = *reinterpret_cast<const __nv_bfloat162*>(&w);
-                    const float2 f = __bfloat1622float2(hb);
-                    p_lo[i] = Cvt<T>::pack(a - f.x, c - f.y);
-                }
-            }
-            // (e) The P slot must be free before it is overwritten.
-            if (t >= kPLag) confirm_pv(t - kPLag);
-            fence_after_sync();
-            const uint32_t p_col = t_lane + kStreamPCol + (kParts == 2 ? 0u : static_cast<uint32_t>((t & 1) * 32));
-            tmem_st32(p_col, p_hi);
-            if constexpr (kParts == 2) tmem_st32(p_col + 32, p_lo);
-            tmem_wait_st();
-        } else if (t >= kPLag) {
-            confirm_pv(t - kPLag);
-        }
-        // (f) Refill: the stage of tile x is free once Q K^T(x) and P V(x) are
-        // done, which holds for x <= t - kPLag (confirmed above).
-        if (issued < nt && issued - kStages <= t - kPLag) {
-            load_kv(issued);
-            ++issued;
-        }
-        fence_before_sync();
-        __syncthreads();
-        if (s_fail) break;
-        if (tid == 0) {
-            fence_after_sync();
-            const uint32_t p_addr = tmem + kStreamPCol + (kParts == 2 ? 0u : static_cast<uint32_t>((t & 1) * 32));
-#pragma unroll
-            for (int part = 0; part < kParts; ++part)
+                    for (int ks = 0; ks < 4; ++ks)
+                        mma_f16_ts(tmem + kStreamOCol, p_addr + part * 32 + ks * 8,
+                                   make_sdesc(stage_v(t) + ks * 2048), idesc_pv,
+                                   (t > 0 || part > 0 || ks > 0) ? 1u : 0u);
+                mma_commit(pv_done0 + 8 * (t & 1));
+            };
+            for (int t = 0; t < nt && !s_fail; ++t) {
+                // Q K^T(t): the tile has landed, and S buffer t & 1 was released by
+                // p_ready(t - 2), which issue_pv(t - 2) has already waited for.
+                wait_event(kv_ready0 + 8 * (t % kStages), (t / kStages) & 1);
+                fence_after_sync();
+                const uint32_t d = tmem + static_cast<uint32_t>((t & 1) * kTileN);
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
-                    mma_f16_ts(tmem + kStreamOCol, p_addr + part * 32 + ks * 8, make_sdesc(stage_v(t) + ks * 2048),
-                               idesc_pv, (t > 0 || part > 0 || ks > 0) ? 1u : 0u);
-            mma_commit(mbar0 + 16 + 8 * (t & 1));
+                    mma_f16(d, make_sdesc(sQ + ks * 32), make_sdesc(stage_k(t) + ks * 32), idesc_qk, ks > 0);
+                mma_commit(s_ready0 + 8 * (t & 1));
+                if (t >= 1) issue_pv(t - 1);
+            }
+            if (!s_fail) issue_pv(nt - 1);
         }
-    }
+    } else {
+        // ---------------- loads + softmax (one thread per query row) ----------------
+        const uint32_t t_lane = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+        const int row = q0 + tid;
+        const bool warp_rows = q0 + warp * 32 < len;
+        constexpr int kPLag = kParts == 2 ? 1 : 2;
+        int pv_seen = -1;
+        auto confirm_pv = [&](int x) {
+            if (x > pv_seen) {
+                wait_event(pv_done0 + 8 * (x & 1), (x >> 1) & 1);
+                pv_seen = x;
+            }
+        };
+        // Publish tile t (its copies, and every earlier group, have landed).
+        auto publish = [&](int t) {
+            resident::cp_async_wait_pending(issued - 1 - t);
+            fence_async_smem();
+            arrive(kv_ready0 + 8 * (t % kStages));
+        };
+        publish(0);
 
-    // Epilogue: wait for the last product, O / l.
-    if (!s_fail) {
-        confirm_pv(nt - 1);
-        if (!s_fail && warp_rows) {
+        float m_ref = -INFINITY;   // reference maximum (log2 units) of this row
+        float l = 0.f;
+        for (int t = 0; t < nt; ++t) {
+            if (s_fail) break;
+            // Refill the ring: the stage of tile x is free once P V(x) is done.
+            if (issued < nt && issued - kStages <= t - kPLag) {
+                if (t >= kPLag) confirm_pv(t - kPLag);
+                load_kv(issued);
+                ++issued;
+            }
+            // Let the MMA warp start Q K^T(t + 1) while this tile's softmax runs.
+            if (t + 1 < nt) publish(t + 1);
+
+            wait_event(s_ready0 + 8 * (t & 1), (t >> 1) & 1);
             fence_after_sync();
-            const float inv = 1.f / l;
-            float v[64];
-            tmem_ld64(t_lane + kStreamOCol, v);
-            uint32_t w[32];
+            const int valid = min(kTileN, len - t * kTileN);
+            if (warp_rows) {
+                float sv[64];
+                tmem_ld64(t_lane + static_cast<uint32_t>((t & 1) * kTileN), sv);
+                if (valid < kTileN) {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) w[i] = Cvt<T>::pack(v[2 * i] * inv, v[2 * i + 1] * inv);
-            if (row < len) {
-                uint4* dst = reinterpret_cast<uint4*>(out + static_cast<int64_t>(start + row) * out_tok_stride +
-                                                      h * 64);
+                    for (int i = 0; i < 64; ++i)
+                        if (i >= valid) sv[i] = -INFINITY;
+                }
+                float mx = -INFINITY;
 #pragma unroll
-                for (int c = 0; c < 8; ++c) dst[c] = make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
-                if (row == 0 && cls_out != nullptr) {
-                    uint4* cd = reinterpret_cast<uint4*>(cls_out + (static_cast<int64_t>(b) * H + h) * 64);
+                for (int i = 0; i < 64; ++i) mx = fmaxf(mx, sv[i]);
+                // Rescale only when the tile's maximum exceeds the reference by
+                // more than the threshold (always for the first tile).
+                const float mt = mx * scale_log2;
+                const bool grow = mt > m_ref + kRescaleThreshold;
+                float alpha = 1.f;
+                if (grow) {
+                    alpha = fast_exp2_guard(m_ref - mt);
+                    l *= alpha;
+                    m_ref = mt;
+                }
+                if (t > 0 && __any_sync(0xffffffffu, grow)) {
+                    // O must hold the finished products of tiles 0 .. t - 1.
+                    confirm_pv(t - 1);
+                    fence_after_sync();
+                    float ov[64];
+                    tmem_ld64(t_lane + kStreamOCol, ov);
 #pragma unroll
-                    for (int c = 0; c < 8; ++c) cd[c] = make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+                    for (int g = 0; g < 4; ++g) {
+                        float part[16];
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) part[i] = ov[g * 16 + i] * alpha;
+                        tmem_st16(t_lane + kStreamOCol + g * 16, part);
+                    }
+                }
+                uint32_t p_hi[32], p_lo[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const float a = mma_attn::fast_exp2(fmaf(sv[2 * i], scale_log2, -m_ref));   // -inf -> 0
+                    const float c = mma_attn::fast_exp2(fmaf(sv[2 * i + 1], scale_log2, -m_ref));
+                    l += a + c;
+                    const uint32_t w = Cvt<T>::pack(a, c);
+                    p_hi[i] = w;
+                    if constexpr (kParts == 2) {
+                        __nv_bfloat162 hb = *reinterpret_cast<const __nv_bfloat162*>(&w);
+                        const float2 f = __bfloat1622float2(hb);
+                        p_lo[i] = Cvt<T>::pack(a - f.x, c - f.y);
+                    }
+                }
+                // The P slot is free once the product that last read it is done.
+                if (t >= kPLag) confirm_pv(t - kPLag);
+                fence_after_sync();
+                const uint32_t p_col = t_lane + kStreamPCol + (kParts == 2 ? 0u : static_cast<uint32_t>((t & 1) * 32));
+                tmem_st32(p_col, p_hi);
+                if constexpr (kParts == 2) tmem_st32(p_col + 32, p_lo);
+                tmem_wait_st();
+            }
+            fence_before_sync();
+            arrive(p_ready0 + 8 * (t & 1));
+        }
+
+        // Epilogue: wait for the last product, O / l.
+        if (!s_fail) {
+            confirm_pv(nt - 1);
+            if (!s_fail && warp_rows) {
+                fence_after_sync();
+                const float inv = 1.f / l;
+                float v[64];
+                tmem_ld64(t_lane + kStreamOCol, v);
+                uint32_t w[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) w[i] = Cvt<T>::pack(v[2 * i] * inv, v[2 * i + 1] * inv);
+                if (row < len) {
+                    uint4* dst = reinterpret_cast<uint4*>(out + static_cast<int64_t>(start + row) * out_tok_stride +
+                                                          h * 64);
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) dst[c] = make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+                    if (row == 0 && cls_out != nullptr) {
+                        uint4* cd = reinterpret_cast<uint4*>(cls_out + (static_cast<int64_t>(b) * H + h) * 64);
+#pragma unroll
+                        for (int c = 0; c < 8; ++c)
+                            cd[c] = make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+                    }
                 }
             }
         }
+        cp_async_wait<0>();
     }
 
-    cp_async_wait<0>();
     fence_before_sync();
     __syncthreads();
     if (s_fail && tid == 0) raise_status(RAGGED_DEV_TIMEOUT);

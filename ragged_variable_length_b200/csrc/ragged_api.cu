@@ -148,7 +148,7 @@ ragged_status launch_tc05(const ragged::resident::PackedRows& src, int64_t B, in
     if (st != RAGGED_OK) return st;
     const dim3 grid(static_cast<unsigned>((max_seqlen + kRows - 1) / kRows), static_cast<unsigned>(H),
                     static_cast<unsigned>(B));
-    kernel<<<grid, kThreads, smem, s>>>(src, scale * 1.4426950408889634f, static_cast<int>(H),
+    kernel<<<grid, kStreamThreads, smem, s>>>(src, scale * 1.4426950408889634f, static_cast<int>(H),
                                         static_cast<uint16_t*>(out), out_tok_stride, static_cast<uint16_t*>(cls_out));
     return cuda_check(cudaGetLastError(), "tcgen05 attention launch");
 }
