@@ -433,7 +433,7 @@ def run_ours(args, rank, world, dist):
             t_roof = max(bts / (hbm_peak * 1e9), fl / (bf16_peak * 1e12))
             per_kernel = {}
             for kname, kcode in (("streaming", rv.RAGGED_ATTN_STREAMING), ("resident", rv.RAGGED_ATTN_RESIDENT),
-                                 ("tcgen05", rv.RAGGED_ATTN_TCGEN05)):
+                                 ("tcgen05", rv.RAGGED_ATTN_TCGEN05), ("persistent", rv.RAGGED_ATTN_PERSISTENT)):
                 prev = rv.ragged_set_attn_kernel(kcode)
                 try:
                     t = graph_time([attn_launcher(p_, w_) for p_, w_ in zip(pls, ws)], replays=max(3, 30 // copies))
@@ -572,15 +572,17 @@ def run_reference(args, rank, world):
     }), flush=True)
 
 
-PROFILE_CASES = ("serving", "hires")
+PROFILE_CASES = ("serving", "hires", "sweep")
 
 
 def run_profile_case(case: str) -> None:
     """One untimed pass of a workload, for an ncu capture of its kernels.
 
     serving: the fused pipeline once on each of the 12 serving batches.
-    hires:   the 384x384 B=64 workload packed, then attention twice with the
-             streaming mma.sync kernel and twice with the tcgen05 kernel.
+    hires:   the 384x384 B=64 workload packed, then attention twice with each
+             of the streaming mma.sync, tcgen05 and persistent tcgen05 kernels.
+    sweep:   the B=512, 0% pruning sweep workload packed, then attention twice
+             with each of the same three kernels.
     """
     import torch
     import ragged_variable_length_b200 as rv
@@ -596,12 +598,13 @@ def run_profile_case(case: str) -> None:
         torch.cuda.synchronize()
         for pl in pls:
             pl()
-    elif case == "hires":
-        w = synthetic.hires_384()
-        pl = rv.Pipeline(w.B, w.L_full, w.H, torch.bfloat16, flags=rv.RAGGED_PIPELINE_SPLIT)
+    elif case in ("hires", "sweep"):
+        w = synthetic.hires_384() if case == "hires" else synthetic.sweep(0.0)
+        dt = torch.bfloat16 if w.dtype == "bf16" else torch.float16
+        pl = rv.Pipeline(w.B, w.L_full, w.H, dt, flags=rv.RAGGED_PIPELINE_SPLIT)
         pl.dense_qkv.view(torch.int16).copy_(torch.from_numpy(w.qkv.view(np.int16)))
         pl.keep.copy_(torch.from_numpy(w.keep))
-        for kern in (rv.RAGGED_ATTN_STREAMING, rv.RAGGED_ATTN_TCGEN05):
+        for kern in (rv.RAGGED_ATTN_STREAMING, rv.RAGGED_ATTN_TCGEN05, rv.RAGGED_ATTN_PERSISTENT):
             rv.ragged_set_attn_kernel(kern)
             pl()
             pl()

@@ -143,12 +143,15 @@ RAGGED_API ragged_status ragged_attn_fwd(const void *q, const void *k, const voi
                               void *cls_out, void *stream);
 
 /* Attention kernels (ragged_set_attn_kernel). */
-#define RAGGED_ATTN_AUTO 0      /* per launch shape (default): RESIDENT for launches too small
-                                   to fill the GPU or single-tile sequences, TCGEN05 for
-                                   max_seqlen above 256, STREAMING otherwise               */
-#define RAGGED_ATTN_STREAMING 1 /* mma.sync, K/V tiles streamed, any max_seqlen             */
-#define RAGGED_ATTN_RESIDENT 2  /* mma.sync, whole sequence in shared memory, <= 640 keys  */
-#define RAGGED_ATTN_TCGEN05 3   /* tcgen05.mma with TMEM accumulators, K/V streamed        */
+#define RAGGED_ATTN_AUTO 0       /* per launch shape (default): RESIDENT for launches too
+                                    small to fill the GPU or single-tile sequences,
+                                    PERSISTENT for long sequences, STREAMING otherwise    */
+#define RAGGED_ATTN_STREAMING 1  /* mma.sync, K/V tiles streamed, any max_seqlen            */
+#define RAGGED_ATTN_RESIDENT 2   /* mma.sync, whole sequence in shared memory, <= 640 keys */
+#define RAGGED_ATTN_TCGEN05 3    /* tcgen05.mma with TMEM accumulators, K/V streamed, one
+                                    CTA per (128-query tile, head, sequence)               */
+#define RAGGED_ATTN_PERSISTENT 4 /* tcgen05.mma, persistent CTAs with a TMA load warp;
+                                    B <= 1024 (larger B runs RAGGED_ATTN_TCGEN05)          */
 
 /*
  * ragged_set_attn_kernel - process-wide choice of the f16/bf16 attention

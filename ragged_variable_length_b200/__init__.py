@@ -42,6 +42,7 @@ RAGGED_ATTN_AUTO = 0
 RAGGED_ATTN_STREAMING = 1
 RAGGED_ATTN_RESIDENT = 2
 RAGGED_ATTN_TCGEN05 = 3
+RAGGED_ATTN_PERSISTENT = 4
 
 DTYPE_CODES = {torch.float16: 0, torch.bfloat16: 1, torch.float32: 2}
 DTYPE_NAMES = {"f16": torch.float16, "bf16": torch.bfloat16, "f32": torch.float32}

@@ -1,0 +1,577 @@
+// Persistent, warp-specialised ragged attention on the 5th-generation tensor
+// cores (tcgen05.mma with TMEM accumulators, TMA loads), f16 / bf16,
+// head_dim 64.
+//
+// Operation ("Dispatch-Aware Ragged Attention for Pruned Vision Transformers",
+// abstract; radpulse section "Bypassing the binding"): per sequence b and head
+// h, O = softmax(scale Q K^T) V over the sequence's own rows, no causal mask,
+// no padding.
+//
+// Work items are (sequence, 128-query tile, head) triples, numbered densely.
+// Each CTA copies cu_seqlens into shared memory once, forms the exclusive
+// prefix of H * ceil(L_b / 128) over the sequences, and takes items
+// blockIdx.x, blockIdx.x + gridDim.x, ...; two CTAs share an SM.  TMEM
+// (256 columns: S of two tiles, P, O) and the mbarriers are set up once per
+// CTA, so the per-launch fixed costs of a CTA (cu_seqlens read, TMEM
+// allocation, first loads) are paid once, and the loads of the next item run
+// under the softmax of the current one.
+//
+// Warp roles; they hand off through mbarriers only:
+//   warp 5     loads.  Full tiles by TMA from 3-D tensor maps over
+//              [rows, head, 64] with the 128-byte swizzle, which is the
+//              canonical SWIZZLE_128B operand layout of tcgen05; partial tiles
+//              (the last rows of a sequence) by cp.async with zero fill, their
+//              completion signalled by cp.async.mbarrier.arrive.noinc.  Q is
+//              double-buffered, K/V flow through a 4-stage ring.
+//   warp 4     one thread issues every tcgen05.mma: S = Q K^T of tile g into
+//              TMEM buffer g & 1 as soon as the tile has landed, then P V of
+//              tile g - 1 (P read from TMEM, V from shared memory).  An
+//              item's last P V is issued before the next item's first Q K^T.
+//   warps 0-3  softmax, one thread per query row (TMEM lane = row), single
+//              pass with a reference maximum that is raised (and the running
+//              sum and O rescaled) only when a tile exceeds it by more than
+//              2^8; P goes to TMEM (bf16: hi and lo parts).  The pairwise
+//              fp32 work uses the packed f32x2 instructions of sm_100.  The
+//              epilogue reads O from TMEM, releases it to the next item, and
+//              stores O / l (and the CLS row).
+// The tile counter g runs across items, so every buffer parity carries over
+// from one item to the next.
+//
+// Every mbarrier wait is bounded; a wait that gives up sets RAGGED_DEV_TIMEOUT
+// in the status word, every role leaves its loop, the MMA thread waits for its
+// own MMAs and the load warp for its own copies, and TMEM is freed.
+#pragma once
+
+#include <cuda.h>
+
+#include "attn_tc05.cuh"
+
+namespace ragged {
+namespace tc05 {
+
+constexpr int kPersistThreads = 192;
+constexpr int kPersistStages = 4;
+constexpr int kPersistMaxB = 1024;   // cu_seqlens and item offsets live in shared memory
+constexpr int kMmaWarp = 4;
+constexpr int kLoadWarp = 5;
+constexpr uint32_t kFullMask = 0xffffffffu;
+
+// Dynamic shared memory: alignment slack, two Q buffers, the K/V ring, then
+// cu_seqlens and the item offsets (B + 1 ints each).
+__host__ __device__ constexpr int persist_smem_bytes(int B) {
+    return 1024 + 2 * kQBytes + kPersistStages * 2 * kKVTileBytes + 2 * (B + 1) * 4;
+}
+
+struct PersistArgs {
+    const uint16_t* q;
+    const uint16_t* k;
+    const uint16_t* v;
+    int64_t tok_stride, head_stride;   // elements
+    const int32_t* cu;
+    int B, H, max_seqlen;
+    float scale_log2;
+    uint16_t* out;
+    int64_t out_tok_stride;
+    uint16_t* cls_out;
+};
+
+// ---- mbarrier, TMA and packed-fp32 wrappers --------------------------------
+
+__device__ __forceinline__ void mbar_arrive(uint32_t mbar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(mbar) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t mbar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(mbar), "r"(bytes) : "memory");
+}
+// Arrives on mbar once every cp.async this thread has issued so far has landed.
+__device__ __forceinline__ void cp_async_arrive_noinc(uint32_t mbar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(mbar) : "memory");
+}
+// One box of a 3-D tensor map (coordinates innermost first) into shared
+// memory, completing `bytes` of the transaction count of mbar.
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int x, int y, int z,
+                                            uint32_t mbar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
+        "[%5];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(mbar)
+        : "memory");
+}
+__device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+__device__ __forceinline__ uint64_t f2(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f2_split(uint64_t v, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+// 32 consecutive fp32 columns of this thread's TMEM lane, one load and its wait.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,"
+        "%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n\t"
+        "tcgen05.wait::ld.sync.aligned;\n"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr)
+        : "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+// 16 consecutive 32-bit TMEM columns of this thread's lane <- v (no wait).
+__device__ __forceinline__ void tmem_st16_u(uint32_t taddr, const uint32_t (&v)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};\n"
+        :
+        : "r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+          "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+        : "memory");
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+// Rows [row0, row0 + ROWS) of one head of a sequence (base = its row 0) into a
+// swizzled tile by the 32 lanes of a warp; rows at or past len are zero-filled
+// without being read.
+template <int ROWS>
+__device__ __forceinline__ void warp_load_rows(uint32_t s_tile, const uint16_t* base, int64_t tok_stride, int row0,
+                                               int len, int lane) {
+#pragma unroll 4
+    for (int i = lane; i < ROWS * 8; i += 32) {
+        const int r = i >> 3, c = i & 7;
+        const int row = row0 + r;
+        const bool ok = row < len;
+        cp_async_16(s_tile + swz(r, c), base + static_cast<int64_t>(ok ? row : 0) * tok_stride + c * 8, ok ? 16 : 0);
+    }
+}
+
+struct Item {
+    int h, q0, start, len, nt, b;
+};
+
+// Item j -> (sequence, query tile, head); s_ip holds the exclusive item
+// prefix over sequences (s_ip[B] = number of items > j).
+__device__ __forceinline__ Item decode_item(int j, const int* s_cu, const int* s_ip, int B, int H) {
+    int lo = 0, hi = B;   // s_ip[lo] <= j < s_ip[hi]
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (s_ip[mid] <= j) lo = mid;
+        else hi = mid;
+    }
+    Item it;
+    it.b = lo;
+    const int r = j - s_ip[lo];
+    const int qt = r / H;
+    it.h = r - qt * H;
+    it.q0 = qt * kRows;
+    it.start = s_cu[lo];
+    it.len = s_cu[lo + 1] - it.start;
+    it.nt = (it.len + kTileN - 1) / kTileN;
+    return it;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kPersistThreads, 2)
+    attn_tc05_persist_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                             const __grid_constant__ CUtensorMap tm_v, const PersistArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    // kv_full[S], kv_empty[S], q_full[2], q_empty[2], s_full[2], p_full[2], pv_done[2], o_empty, drain
+    __shared__ __align__(8) uint64_t s_bar[2 * kPersistStages + 12];
+    __shared__ uint32_t s_tmem;
+    __shared__ int s_fail;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    constexpr int S = kPersistStages;
+    constexpr int kParts = Cvt<T>::kParts;
+
+    const uint32_t raw = smem_addr(smem_raw);
+    const uint32_t sQ = (raw + 1023u) & ~1023u;   // Q buffer i at sQ + i * 16 KB
+    const uint32_t sRing = sQ + 2 * kQBytes;      // stage s: K at sRing + s * 16 KB, V 8 KB further
+    int* s_cu = reinterpret_cast<int*>(smem_raw + (sRing - raw) + S * 2 * kKVTileBytes);
+    int* s_ip = s_cu + (a.B + 1);
+
+    const uint32_t bar0 = smem_addr(&s_bar[0]);
+    auto kv_full = [&](int s) { return bar0 + 8u * s; };
+    auto kv_empty = [&](int s) { return bar0 + 8u * (S + s); };
+    auto q_full = [&](int i) { return bar0 + 8u * (2 * S + i); };
+    auto q_empty = [&](int i) { return bar0 + 8u * (2 * S + 2 + i); };
+    auto s_full = [&](int i) { return bar0 + 8u * (2 * S + 4 + i); };
+    auto p_full = [&](int i) { return bar0 + 8u * (2 * S + 6 + i); };
+    auto pv_done = [&](int i) { return bar0 + 8u * (2 * S + 8 + i); };
+    const uint32_t o_empty = bar0 + 8u * (2 * S + 10);
+    const uint32_t drain = bar0 + 8u * (2 * S + 11);
+    volatile int* fail_flag = &s_fail;
+
+    // ---- setup: cu_seqlens, barriers, TMEM, item offsets ----
+    for (int i = tid; i <= a.B; i += kPersistThreads) s_cu[i] = __ldg(a.cu + i);
+    if (tid == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(kv_full(s), 32);
+            mbar_init(kv_empty(s), 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(q_full(i), 32);
+            mbar_init(q_empty(i), 1);
+            mbar_init(s_full(i), 1);
+            mbar_init(p_full(i), kSoftmaxThreads);
+            mbar_init(pv_done(i), 1);
+        }
+        mbar_init(o_empty, kSoftmaxThreads);
+        mbar_init(drain, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        s_fail = 0;
+    }
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(&s_tmem)),
+                     "r"(kStreamTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    if (warp == kLoadWarp && lane == 0) {
+        prefetch_tensormap(&tm_q);
+        prefetch_tensormap(&tm_k);
+        prefetch_tensormap(&tm_v);
+    }
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    if (warp == kLoadWarp) {   // item offsets: warp-wide inclusive scans over 32 sequences at a time
+        int carry = 0;
+        if (lane == 0) s_ip[0] = 0;
+        for (int c0 = 0; c0 < a.B; c0 += 32) {
+            const int b = c0 + lane;
+            int n = 0;
+            if (b < a.B) {
+                const int st = s_cu[b], len = s_cu[b + 1] - st;
+                if (st < 0 || len < 0 || len > a.max_seqlen) raise_status(RAGGED_DEV_BAD_SEQLENS);
+                else n = ((len + kRows - 1) / kRows) * a.H;
+            }
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(kFullMask, n, o);
+                if (lane >= o) n += y;
+            }
+            if (b < a.B) s_ip[b + 1] = carry + n;
+            carry += __shfl_sync(kFullMask, n, 31);
+        }
+    }
+    __syncthreads();
+    const int total = s_ip[a.B];
+    const uint32_t tmem = s_tmem;
+
+    if (warp == kLoadWarp) {
+        // ---------------- loads ----------------
+        // Warp-uniform bounded wait (every lane acquires the barrier).
+        auto warp_wait = [&](uint32_t mbar, uint32_t parity) {
+            const bool ok = __all_sync(kFullMask, mbar_wait(mbar, parity));
+            if (!ok && lane == 0) atomicExch(&s_fail, 1);
+            return ok;
+        };
+        uint32_t g = 0;
+        int k = 0;
+        bool ok = true;
+        for (int j = blockIdx.x; ok && j < total; j += gridDim.x, ++k) {
+            if (__any_sync(kFullMask, *fail_flag != 0)) break;
+            const Item it = decode_item(j, s_cu, s_ip, a.B, a.H);
+            const int64_t seq_off = static_cast<int64_t>(it.start) * a.tok_stride +
+                                    static_cast<int64_t>(it.h) * a.head_stride;
+            const int qb = k & 1;
+            if (k >= 2 && !warp_wait(q_empty(qb), ((k >> 1) - 1) & 1)) break;
+            const uint32_t sq = sQ + qb * kQBytes;
+            if (it.q0 + kRows <= it.len) {
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(q_full(qb), kQBytes);
+                    tma_load_3d(sq, &tm_q, 0, it.h, it.start + it.q0, q_full(qb));
+                } else {
+                    mbar_arrive(q_full(qb));
+                }
+            } else {
+                warp_load_rows<kRows>(sq, a.q + seq_off, a.tok_stride, it.q0, it.len, lane);
+                cp_async_arrive_noinc(q_full(qb));
+            }
+            for (int t = 0; t < it.nt; ++t, ++g) {
+                const int s = static_cast<int>(g % S);
+                if (g >= static_cast<uint32_t>(S) && !warp_wait(kv_empty(s), ((g / S) - 1) & 1)) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t sk = sRing + s * 2 * kKVTileBytes;
+                const int r0 = t * kTileN;
+                if (r0 + kTileN <= it.len) {
+                    if (lane == 0) {
+                        mbar_arrive_expect_tx(kv_full(s), 2 * kKVTileBytes);
+                        tma_load_3d(sk, &tm_k, 0, it.h, it.start + r0, kv_full(s));
+                        tma_load_3d(sk + kKVTileBytes, &tm_v, 0, it.h, it.start + r0, kv_full(s));
+                    } else {
+                        mbar_arrive(kv_full(s));
+                    }
+                } else {
+                    warp_load_rows<kTileN>(sk, a.k + seq_off, a.tok_stride, r0, it.len, lane);
+                    warp_load_rows<kTileN>(sk + kKVTileBytes, a.v + seq_off, a.tok_stride, r0, it.len, lane);
+                    cp_async_arrive_noinc(kv_full(s));
+                }
+            }
+        }
+        cp_async_wait<0>();
+        if (*fail_flag) {
+            // Let the TMA loads still in flight land before the CTA can exit:
+            // the newest tile of each ring stage and the newest Q loads.
+            for (uint32_t x = g > static_cast<uint32_t>(S) ? g - S : 0; x < g; ++x) mbar_wait(kv_full(x % S), (x / S) & 1);
+            for (int x = k > 2 ? k - 2 : 0; x < k; ++x) mbar_wait(q_full(x & 1), (x >> 1) & 1);
+        }
+    } else if (warp == kMmaWarp) {
+        // ---------------- MMA issue (one thread) ----------------
+        if (lane == 0) {
+            const uint32_t idesc_qk = make_idesc(Cvt<T>::kFormat, 0, kTileN);
+            const uint32_t idesc_pv = make_idesc(Cvt<T>::kFormat, 1, 64);
+            // P V of tile x (the first of its item when `first`, item index kk).
+            auto issue_pv = [&](uint32_t x, bool first, int kk) {
+                if (!mbar_wait(p_full(x & 1), (x >> 1) & 1)) return false;
+                if (first && kk >= 1 && !mbar_wait(o_empty, (kk - 1) & 1)) return false;
+                fence_after_sync();
+                const uint32_t p_addr = tmem + kStreamPCol + (kParts == 2 ? 0u : (x & 1) * 32u);
+                const uint32_t sv = sRing + (x % S) * 2 * kKVTileBytes + kKVTileBytes;
+#pragma unroll
+                for (int part = 0; part < kParts; ++part)
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)
+                        mma_f16_ts(tmem + kStreamOCol, p_addr + part * 32 + ks * 8, make_sdesc(sv + ks * 2048),
+                                   idesc_pv, (first && part == 0 && ks == 0) ? 0u : 1u);
+                mma_commit(pv_done(x & 1));
+                mma_commit(kv_empty(x % S));
+                return true;
+            };
+            uint32_t g = 0;
+            int k = 0;
+            bool ok = true;
+            for (int j = blockIdx.x; ok && j < total; j += gridDim.x, ++k) {
+                const Item it = decode_item(j, s_cu, s_ip, a.B, a.H);
+                const int qb = k & 1;
+                if (!mbar_wait(q_full(qb), (k >> 1) & 1)) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t sq = sQ + qb * kQBytes;
+                for (int t = 0; t < it.nt; ++t, ++g) {
+                    const int s = static_cast<int>(g % S);
+                    if (!mbar_wait(kv_full(s), (g / S) & 1)) {
+                        ok = false;
+                        break;
+                    }
+                    // Tiles filled by cp.async were written through the generic
+                    // proxy; order them before the tensor core's reads.
+                    fence_async_smem();
+                    fence_after_sync();
+                    const uint32_t d = tmem + (g & 1) * static_cast<uint32_t>(kTileN);
+                    const uint32_t sk = sRing + s * 2 * kKVTileBytes;
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)
+                        mma_f16(d, make_sdesc(sq + ks * 32), make_sdesc(sk + ks * 32), idesc_qk, ks > 0);
+                    mma_commit(s_full(g & 1));
+                    if (t == it.nt - 1) mma_commit(q_empty(qb));
+                    if (t >= 1 && !issue_pv(g - 1, t == 1, k)) {
+                        ok = false;
+                        break;
+                    }
+                }
+                if (ok && !issue_pv(g - 1, it.nt == 1, k)) ok = false;
+            }
+            if (!ok) atomicExch(&s_fail, 1);
+            // Every MMA this thread issued has completed before TMEM is freed.
+            mma_commit(drain);
+            mbar_wait(drain, 0);
+        }
+    } else {
+        // ---------------- softmax and epilogue (one thread per query row) ----------------
+        const uint32_t t_lane = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+        constexpr int kPLag = kParts == 2 ? 1 : 2;   // P slots: bf16 one (hi + lo), f16 two
+        int pv_seen = -1;
+        auto confirm_pv = [&](int x) {
+            if (x > pv_seen) {
+                if (!mbar_wait(pv_done(x & 1), (x >> 1) & 1)) atomicExch(&s_fail, 1);
+                pv_seen = x;
+            }
+        };
+        const uint64_t sl2 = f2(a.scale_log2, a.scale_log2);
+        int g = 0;
+        int k = 0;
+        for (int j = blockIdx.x; j < total; j += gridDim.x, ++k) {
+            if (*fail_flag) break;
+            const Item it = decode_item(j, s_cu, s_ip, a.B, a.H);
+            const int row = it.q0 + tid;
+            const bool warp_rows = it.q0 + warp * 32 < it.len;
+            float m_ref = -INFINITY;   // reference maximum (log2 units) of this row
+            float l0 = 0.f, l1 = 0.f;  // running sum, even / odd keys
+            bool ok = true;
+            for (int t = 0; t < it.nt; ++t, ++g) {
+                if (!mbar_wait(s_full(g & 1), (g >> 1) & 1)) {
+                    atomicExch(&s_fail, 1);
+                    ok = false;
+                    break;
+                }
+                fence_after_sync();
+                if (warp_rows) {
+                    float sv[64];
+                    tmem_ld64(t_lane + static_cast<uint32_t>((g & 1) * kTileN), sv);
+                    const int valid = min(kTileN, it.len - t * kTileN);
+                    if (valid < kTileN) {
+#pragma unroll
+                        for (int i = 0; i < 64; ++i)
+                            if (i >= valid) sv[i] = -INFINITY;
+                    }
+                    float mq[4];
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        float m = fmax3(sv[16 * c], sv[16 * c + 1], sv[16 * c + 2]);
+#pragma unroll
+                        for (int i = 3; i < 15; i += 2) m = fmax3(m, sv[16 * c + i], sv[16 * c + i + 1]);
+                        mq[c] = fmaxf(m, sv[16 * c + 15]);
+                    }
+                    const float mt = fmaxf(fmax3(mq[0], mq[1], mq[2]), mq[3]) * a.scale_log2;
+                    // Raise the reference only when the tile's maximum exceeds it
+                    // by more than the threshold (always on the first tile).
+                    const bool grow = mt > m_ref + kRescaleThreshold;
+                    float alpha = 1.f;
+                    if (grow) {
+                        alpha = mma_attn::fast_exp2(m_ref - mt);
+                        l0 *= alpha;
+                        l1 *= alpha;
+                        m_ref = mt;
+                    }
+                    if (t > 0 && __any_sync(kFullMask, grow)) {
+                        // O holds the finished products of this item's tiles so far.
+                        confirm_pv(g - 1);
+                        fence_after_sync();
+                        // 16 columns at a time: sv is still live here.
+                        const uint64_t a2 = f2(alpha, alpha);
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            float part[16];
+                            tmem_ld16(t_lane + kStreamOCol + q * 16, part);
+#pragma unroll
+                            for (int i = 0; i < 8; ++i)
+                                f2_split(f2_mul(f2(part[2 * i], part[2 * i + 1]), a2), part[2 * i], part[2 * i + 1]);
+                            tmem_st16(t_lane + kStreamOCol + q * 16, part);
+                        }
+                    }
+                    // The P slot is free once the product that last read it is done.
+                    if (g >= kPLag) confirm_pv(g - kPLag);
+                    fence_after_sync();
+                    const uint32_t p_col =
+                        t_lane + kStreamPCol + (kParts == 2 ? 0u : static_cast<uint32_t>((g & 1) * 32));
+                    const uint64_t nm = f2(-m_ref, -m_ref);
+                    uint64_t lsum = f2(l0, l1);
+                    // Two halves of 32 keys, each stored as soon as it is ready.
+#pragma unroll
+                    for (int hf = 0; hf < 2; ++hf) {
+                        uint32_t p_hi[16], p_lo[16];
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            const int c = hf * 16 + i;
+                            float x0, x1;
+                            f2_split(f2_fma(f2(sv[2 * c], sv[2 * c + 1]), sl2, nm), x0, x1);
+                            const float e0 = mma_attn::fast_exp2(x0), e1 = mma_attn::fast_exp2(x1);   // -inf -> 0
+                            const uint64_t e = f2(e0, e1);
+                            lsum = f2_add(lsum, e);
+                            const uint32_t w = Cvt<T>::pack(e0, e1);
+                            p_hi[i] = w;
+                            if constexpr (kParts == 2) {
+                                // bf16 -> fp32 is a 16-bit shift; the residual is rounded again.
+                                float r0, r1;
+                                f2_split(f2_sub(e, f2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u))),
+                                         r0, r1);
+                                p_lo[i] = Cvt<T>::pack(r0, r1);
+                            }
+                        }
+                        tmem_st16_u(p_col + hf * 16, p_hi);
+                        if constexpr (kParts == 2) tmem_st16_u(p_col + 32 + hf * 16, p_lo);
+                    }
+                    f2_split(lsum, l0, l1);
+                    tmem_wait_st();
+                }
+                fence_before_sync();
+                mbar_arrive(p_full(g & 1));
+            }
+            if (!ok || *fail_flag) break;
+
+            // Epilogue: the item's last product, O read out (32 columns at a
+            // time) and stored as O / l, then O released to the next item.
+            confirm_pv(g - 1);
+            fence_after_sync();
+            if (warp_rows) {
+                const bool store = row < it.len;
+                const float inv = 1.f / (l0 + l1);
+                const uint64_t inv2 = f2(inv, inv);
+                uint4* dst = reinterpret_cast<uint4*>(a.out + static_cast<int64_t>(it.start + row) * a.out_tok_stride +
+                                                      it.h * 64);
+                uint4* cd = (row == 0 && a.cls_out != nullptr)
+                                ? reinterpret_cast<uint4*>(a.cls_out + (static_cast<int64_t>(it.b) * a.H + it.h) * 64)
+                                : nullptr;
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf) {
+                    float ov[32];
+                    tmem_ld32(t_lane + kStreamOCol + hf * 32, ov);
+                    uint32_t w[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        float o0, o1;
+                        f2_split(f2_mul(f2(ov[2 * i], ov[2 * i + 1]), inv2), o0, o1);
+                        w[i] = Cvt<T>::pack(o0, o1);
+                    }
+                    if (store) {
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) {
+                            const uint4 val = make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+                            dst[hf * 4 + c] = val;
+                            if (cd != nullptr) cd[hf * 4 + c] = val;
+                        }
+                    }
+                }
+            }
+            fence_before_sync();
+            mbar_arrive(o_empty);
+        }
+    }
+
+    fence_before_sync();
+    __syncthreads();
+    if (*fail_flag && tid == 0) raise_status(RAGGED_DEV_TIMEOUT);
+    if (warp == 0) {
+        fence_after_sync();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kStreamTmemCols)
+                     : "memory");
+    }
+}
+
+}  // namespace tc05
+}  // namespace ragged

@@ -5,6 +5,7 @@
 // (the paper's radpulse section "Bypassing the binding" locates the
 // dispatch floor of FA2's varlen path in argument conversion, output and
 // softmax_lse allocation and the launch itself).
+#include <algorithm>
 #include <cstdarg>
 #include <cstdio>
 #include <type_traits>
@@ -13,7 +14,10 @@
 #include "attn_mma.cuh"
 #include "attn_resident.cuh"
 #include "attn_tc05.cuh"
+#include "attn_tc05_persist.cuh"
 #include <atomic>
+#include <cudaTypedefs.h>
+#include <mutex>
 #include "common.cuh"
 #include "pack.cuh"
 
@@ -153,6 +157,109 @@ ragged_status launch_tc05(const ragged::resident::PackedRows& src, int64_t B, in
     return cuda_check(cudaGetLastError(), "tcgen05 attention launch");
 }
 
+// ---- TMA tensor maps for the persistent kernel ------------------------------
+
+// cuTensorMapEncodeTiled from the driver, found once through the runtime (the
+// library links no driver library of its own).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// Encoded maps are cached by their parameters, so repeated calls on the same
+// buffers encode nothing.
+struct MapKey {
+    const void* ptr;
+    int64_t H, rows, head_stride, tok_stride;
+    int box_rows;
+    bool operator==(const MapKey& o) const {
+        return ptr == o.ptr && H == o.H && rows == o.rows && head_stride == o.head_stride &&
+               tok_stride == o.tok_stride && box_rows == o.box_rows;
+    }
+};
+constexpr int kMapCache = 24;
+struct MapCache {
+    std::mutex mu;
+    MapKey key[kMapCache];
+    CUtensorMap map[kMapCache];
+    int used = 0, next = 0;
+};
+MapCache g_maps;
+
+// 3-D map over one operand of a [rows, H, 64] 16-bit view (token stride and
+// head stride in elements): box = 64 elements x 1 head x box_rows rows with the
+// 128-byte swizzle.  False when the driver rejects the layout.
+bool tensor_map_3d(CUtensorMap* out, const void* ptr, int64_t H, int64_t rows, int64_t head_stride,
+                   int64_t tok_stride, int box_rows) {
+    const MapKey key{ptr, H, rows, head_stride, tok_stride, box_rows};
+    std::lock_guard<std::mutex> lock(g_maps.mu);
+    for (int i = 0; i < g_maps.used; ++i)
+        if (g_maps.key[i] == key) {
+            *out = g_maps.map[i];
+            return true;
+        }
+    PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
+    if (encode == nullptr) return false;
+    const cuuint64_t dims[3] = {64, static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(rows)};
+    // A single head has no head stride of its own; any legal value will do.
+    const int64_t hs = H == 1 ? 64 : head_stride;
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(hs * 2), static_cast<cuuint64_t>(tok_stride * 2)};
+    const cuuint32_t box[3] = {64, 1, static_cast<cuuint32_t>(box_rows)};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    CUtensorMap m;
+    if (encode(&m, CU_TENSOR_MAP_DATA_TYPE_UINT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return false;
+    const int slot = g_maps.used < kMapCache ? g_maps.used++ : (g_maps.next++ % kMapCache);
+    g_maps.key[slot] = key;
+    g_maps.map[slot] = m;
+    *out = m;
+    return true;
+}
+
+bool g_persist_smem[2][kMaxDevices];
+
+// Launches the persistent tcgen05 kernel; *launched = false (and nothing is
+// enqueued) when the launch shape is outside what it supports.
+template <typename T>
+ragged_status launch_tc05_persist(const ragged::resident::PackedRows& src, int64_t B, int64_t H,
+                                  int64_t max_seqlen, float scale, void* out, int64_t out_tok_stride, void* cls_out,
+                                  int slot, cudaStream_t s, bool* launched) {
+    using namespace ragged::tc05;
+    *launched = false;
+    const int64_t q_tiles = (max_seqlen + kRows - 1) / kRows;
+    if (B > kPersistMaxB || B * H * q_tiles >= (int64_t(1) << 31)) return RAGGED_OK;
+    // Full tiles never reach past the last row of their sequence, and every
+    // sequence ends within B * max_seqlen rows.
+    const int64_t rows = B * max_seqlen;
+    CUtensorMap tq, tk, tv;
+    if (!tensor_map_3d(&tq, src.q, H, rows, src.head_stride, src.tok_stride, kRows) ||
+        !tensor_map_3d(&tk, src.k, H, rows, src.head_stride, src.tok_stride, kTileN) ||
+        !tensor_map_3d(&tv, src.v, H, rows, src.head_stride, src.tok_stride, kTileN))
+        return RAGGED_OK;
+    auto kernel = attn_tc05_persist_kernel<T>;
+    ragged_status st = ensure_smem(kernel, persist_smem_bytes(kPersistMaxB), g_persist_smem[slot]);
+    if (st != RAGGED_OK) return st;
+    const int64_t items_bound = B * H * q_tiles;
+    const int64_t ctas = std::min<int64_t>(items_bound, 2LL * sm_count());
+    PersistArgs args{src.q, src.k, src.v, src.tok_stride, src.head_stride, src.cu, static_cast<int>(B),
+                     static_cast<int>(H), static_cast<int>(max_seqlen), scale * 1.4426950408889634f,
+                     static_cast<uint16_t*>(out), out_tok_stride, static_cast<uint16_t*>(cls_out)};
+    kernel<<<static_cast<unsigned>(ctas), kPersistThreads, persist_smem_bytes(static_cast<int>(B)), s>>>(tq, tk, tv,
+                                                                                                        args);
+    *launched = true;
+    return cuda_check(cudaGetLastError(), "persistent tcgen05 attention launch");
+}
+
 // slot: 0/1 packed f16/bf16, 2/3 dense f16/bf16 (one set of smem flags per kernel).
 bool g_res_smem_ks[4][3][kMaxDevices];
 
@@ -180,7 +287,7 @@ extern "C" {
 int32_t ragged_abi_version(void) { return kAbiVersion; }
 
 int32_t ragged_set_attn_kernel(int32_t kernel) {
-    if (kernel < RAGGED_ATTN_AUTO || kernel > RAGGED_ATTN_TCGEN05) return -1;
+    if (kernel < RAGGED_ATTN_AUTO || kernel > RAGGED_ATTN_PERSISTENT) return -1;
     return g_attn_kernel.exchange(kernel);
 }
 
@@ -321,6 +428,16 @@ ragged_status ragged_attn_fwd(const void* q, const void* k, const void* v, int64
     ragged::resident::PackedRows src{static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(k),
                                      static_cast<const uint16_t*>(v), tok_stride, head_stride, cu_seqlens,
                                      static_cast<int>(max_seqlen), 0, 0, 0};
+    if (kernel_choice == RAGGED_ATTN_PERSISTENT) {
+        bool launched = false;
+        st = dtype == RAGGED_F16
+                 ? launch_tc05_persist<__half>(src, B, H, max_seqlen, scale, out, out_tok_stride, cls_out, 0, s,
+                                               &launched)
+                 : launch_tc05_persist<__nv_bfloat16>(src, B, H, max_seqlen, scale, out, out_tok_stride, cls_out, 1,
+                                                      s, &launched);
+        if (st != RAGGED_OK || launched) return st;
+        kernel_choice = RAGGED_ATTN_TCGEN05;
+    }
     if (kernel_choice == RAGGED_ATTN_TCGEN05) {
         if (dtype == RAGGED_F16)
             return launch_tc05<__half>(src, B, H, max_seqlen, scale, out, out_tok_stride, cls_out, 0, s);

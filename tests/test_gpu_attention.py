@@ -19,7 +19,9 @@ pytestmark = pytest.mark.gpu
 
 
 KERNELS = {"auto": rv.RAGGED_ATTN_AUTO, "streaming": rv.RAGGED_ATTN_STREAMING,
-           "resident": rv.RAGGED_ATTN_RESIDENT, "tcgen05": rv.RAGGED_ATTN_TCGEN05}
+           "resident": rv.RAGGED_ATTN_RESIDENT, "tcgen05": rv.RAGGED_ATTN_TCGEN05,
+           "persistent": rv.RAGGED_ATTN_PERSISTENT}
+TC05 = ["tcgen05", "persistent"]
 
 
 def run_pipeline(w, separate_qkv=False, out_pad=0, max_seqlen=None, kernel="auto"):
@@ -114,13 +116,15 @@ def test_kernel_limits_are_reported():
 
 
 @pytest.mark.parametrize("dtype", ["f16", "bf16"])
-def test_long_sequences_tcgen05(dtype):
-    """The tcgen05 kernel streams K/V, so it takes sequences of any length."""
+@pytest.mark.parametrize("kernel", TC05)
+def test_long_sequences_tcgen05(dtype, kernel):
+    """The tcgen05 kernels stream K/V, so they take sequences of any length."""
     w = synthetic.make_workload("long_tc", 4, 1000, 2, [1000, 700, 641, 65], dtype, 83)
-    check_against_oracle(w, kernel="tcgen05")
+    check_against_oracle(w, kernel=kernel)
 
 
-def test_tcgen05_rescale_path():
+@pytest.mark.parametrize("kernel", TC05)
+def test_tcgen05_rescale_path(kernel):
     """Keys whose logits jump by far more than the rescale threshold after the
     first tile force the in-TMEM rescaling of O."""
     w = synthetic.make_workload("jump", 3, 300, 2, [300, 200, 129], "f16", 84)
@@ -131,7 +135,7 @@ def test_tcgen05_rescale_path():
     w.qkv = w.qkv.copy()
     w.qkv[:, :, 0] = q.astype(np.float16)
     w.qkv[:, :, 1] = k.astype(np.float16)
-    check_against_oracle(w, kernel="tcgen05")
+    check_against_oracle(w, kernel=kernel)
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "f16"])
@@ -233,3 +237,57 @@ def test_ragged_pipeline_binding():
     T = int(cu_ref[-1])
     assert np.array_equal(cu.cpu().numpy(), cu_ref)
     assert torch.equal(out[:T], out_ref[:T]) and torch.equal(cls, cls_ref)
+
+
+@pytest.mark.parametrize("kernel", list(KERNELS))
+def test_zero_length_sequences(kernel):
+    """Empty sequences (cu[b] == cu[b + 1]) anywhere in the batch produce no
+    rows and leave their neighbours' results unchanged."""
+    H, d = 3, 64
+    lengths = [0, 70, 0, 0, 129, 1, 0, 64, 0]
+    cu = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+    T = int(cu[-1])
+    rng = synthetic.rng_for(85)
+    qkv = rng.standard_normal((T, 3, H, d)).astype(np.float16)
+    dev = to_device(qkv, "f16")
+    out = torch.full((T + 8, H, d), float("nan"), dtype=torch.float16, device="cuda")
+    cls = torch.full((len(lengths), H, d), 5.0, dtype=torch.float16, device="cuda")
+    rv.ragged_get_device_status()
+    prev = rv.ragged_set_attn_kernel(KERNELS[kernel])
+    try:
+        rv.ragged_attn_fwd(dev[:, 0], dev[:, 1], dev[:, 2], torch.from_numpy(cu).cuda(), 200, 0.125, out=out,
+                           cls_out=cls)
+    finally:
+        rv.ragged_set_attn_kernel(prev)
+    torch.cuda.synchronize()
+    assert rv.ragged_get_device_status() == 0
+    ref = oracle.attention(qkv[:, 0], qkv[:, 1], qkv[:, 2], cu, "f16", 0.125)
+    err, bound = attn_error(to_f64(out[:T]), ref, "f16")
+    assert err <= bound
+    assert torch.isnan(out[T:]).all()
+    for b, L in enumerate(lengths):
+        if L == 0:
+            assert torch.all(cls[b] == 5.0)
+        else:
+            assert torch.equal(cls[b], out[int(cu[b])])
+
+
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+def test_persistent_above_its_batch_limit(dtype):
+    """More sequences than the persistent kernel keeps in shared memory: the
+    launch runs the per-tile tcgen05 kernel instead, with the same results."""
+    rng = np.random.default_rng(86)
+    lengths = rng.integers(1, 80, size=1100)
+    w = synthetic.make_workload("many", 1100, 80, 2, lengths, dtype, 86)
+    check_against_oracle(w, seqs=sample_sequences(w.lengths, 12, seed=3), kernel="persistent")
+
+
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+def test_persistent_many_items_per_cta(dtype):
+    """Several items per CTA with every length class (full and partial query
+    tiles, full and partial key tiles) checked element by element."""
+    rng = np.random.default_rng(87)
+    lengths = rng.integers(1, 400, size=160)
+    lengths[:6] = [1, 64, 128, 129, 256, 399]
+    w = synthetic.make_workload("items", 160, 400, 4, lengths, dtype, 87)
+    check_against_oracle(w, kernel="persistent")
