@@ -20,13 +20,16 @@
 //   warp 5     loads.  Full tiles by TMA from 3-D tensor maps over
 //              [rows, head, 64] with the 128-byte swizzle, which is the
 //              canonical SWIZZLE_128B operand layout of tcgen05; partial tiles
-//              (the last rows of a sequence) by cp.async with zero fill, their
-//              completion signalled by cp.async.mbarrier.arrive.noinc.  Q is
-//              double-buffered, K/V flow through a 4-stage ring.
-//   warp 4     one thread issues every tcgen05.mma: S = Q K^T of tile g into
-//              TMEM buffer g & 1 as soon as the tile has landed, then P V of
-//              tile g - 1 (P read from TMEM, V from shared memory).  An
-//              item's last P V is issued before the next item's first Q K^T.
+//              (the last rows of a sequence) by cp.async with zero fill, each
+//              lane's arrival triggered by the completion of its copies
+//              (cp.async.mbarrier.arrive.noinc).  Q is double-buffered, K/V
+//              flow through a 4-stage ring.
+//   warp 4     one thread issues every tcgen05.mma.  Q K^T runs two tiles
+//              ahead of P V: P V(g) as soon as P(g) is in TMEM, then S of tile
+//              g + 2 into TMEM buffer g & 1, which the softmax has read S(g)
+//              out of.  Across items the walks simply continue, so the next
+//              item's first scores are ready when the current item's
+//              epilogue ends.
 //   warps 0-3  softmax, one thread per query row (TMEM lane = row), single
 //              pass with a reference maximum that is raised (and the running
 //              sum and O rescaled) only when a tile exceeds it by more than
@@ -83,10 +86,6 @@ __device__ __forceinline__ void mbar_arrive(uint32_t mbar) {
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t mbar, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(mbar), "r"(bytes) : "memory");
 }
-// Arrives on mbar once every cp.async this thread has issued so far has landed.
-__device__ __forceinline__ void cp_async_arrive_noinc(uint32_t mbar) {
-    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(mbar) : "memory");
-}
 // One box of a 3-D tensor map (coordinates innermost first) into shared
 // memory, completing `bytes` of the transaction count of mbar.
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int x, int y, int z,
@@ -97,6 +96,12 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
         "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(mbar)
         : "memory");
 }
+// Arrives on mbar once every cp.async this thread has issued so far has landed.
+__device__ __forceinline__ void cp_async_arrive_noinc(uint32_t mbar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(mbar) : "memory");
+}
+// Waits for every cp.async this thread has issued (commits them first).
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -200,13 +205,37 @@ __device__ __forceinline__ Item decode_item(int j, const int* s_cu, const int* s
     return it;
 }
 
+// Cursor over the tiles of a CTA's items: item j (the k-th of this CTA),
+// key tile t of it.
+struct Walk {
+    int j, k, t, total;
+    bool valid;
+    Item it;
+    const int* s_cu;
+    const int* s_ip;
+    int B, H;
+    __device__ __forceinline__ Walk(int j0, int total_, const int* cu, const int* ip, int B_, int H_)
+        : j(j0), k(0), t(0), total(total_), valid(j0 < total_), s_cu(cu), s_ip(ip), B(B_), H(H_) {
+        if (valid) it = decode_item(j, s_cu, s_ip, B, H);
+    }
+    __device__ __forceinline__ void next() {
+        if (++t < it.nt) return;
+        t = 0;
+        ++k;
+        j += gridDim.x;
+        valid = j < total;
+        if (valid) it = decode_item(j, s_cu, s_ip, B, H);
+    }
+};
+
 template <typename T>
 __global__ void __launch_bounds__(kPersistThreads, 2)
     attn_tc05_persist_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                              const __grid_constant__ CUtensorMap tm_v, const PersistArgs a) {
     extern __shared__ uint8_t smem_raw[];
-    // kv_full[S], kv_empty[S], q_full[2], q_empty[2], s_full[2], p_full[2], pv_done[2], o_empty, drain
-    __shared__ __align__(8) uint64_t s_bar[2 * kPersistStages + 12];
+    // kv_full[S], kv_empty[S], q_full[2], q_empty[2], s_full[2], p_full[0..1], pv_done[2], o_empty, drain,
+    // s_free[2], p_full[2..3]
+    __shared__ __align__(8) uint64_t s_bar[2 * kPersistStages + 16];
     __shared__ uint32_t s_tmem;
     __shared__ int s_fail;
 
@@ -226,10 +255,16 @@ __global__ void __launch_bounds__(kPersistThreads, 2)
     auto q_full = [&](int i) { return bar0 + 8u * (2 * S + i); };
     auto q_empty = [&](int i) { return bar0 + 8u * (2 * S + 2 + i); };
     auto s_full = [&](int i) { return bar0 + 8u * (2 * S + 4 + i); };
-    auto p_full = [&](int i) { return bar0 + 8u * (2 * S + 6 + i); };
+    // P of tile g is signalled on p_full(g & 3): warps with no rows in the
+    // current query tile skip the softmax and may arrive for tile g + 2 while
+    // another warp is still working on tile g, so tiles two apart must not
+    // share a barrier (three tiles apart is impossible: Q K^T of tile g + 3
+    // waits until every warp has read S(g + 1)).
+    auto p_full = [&](int i) { return bar0 + 8u * (i < 2 ? 2 * S + 6 + i : 2 * S + 14 + (i - 2)); };
     auto pv_done = [&](int i) { return bar0 + 8u * (2 * S + 8 + i); };
     const uint32_t o_empty = bar0 + 8u * (2 * S + 10);
     const uint32_t drain = bar0 + 8u * (2 * S + 11);
+    auto s_free = [&](int i) { return bar0 + 8u * (2 * S + 12 + i); };
     volatile int* fail_flag = &s_fail;
 
     // ---- setup: cu_seqlens, barriers, TMEM, item offsets ----
@@ -244,7 +279,9 @@ __global__ void __launch_bounds__(kPersistThreads, 2)
             mbar_init(q_empty(i), 1);
             mbar_init(s_full(i), 1);
             mbar_init(p_full(i), kSoftmaxThreads);
+            mbar_init(p_full(i + 2), kSoftmaxThreads);
             mbar_init(pv_done(i), 1);
+            mbar_init(s_free(i), kSoftmaxThreads);
         }
         mbar_init(o_empty, kSoftmaxThreads);
         mbar_init(drain, 1);
@@ -297,6 +334,12 @@ __global__ void __launch_bounds__(kPersistThreads, 2)
             if (!ok && lane == 0) atomicExch(&s_fail, 1);
             return ok;
         };
+        // A partial tile is published without blocking the warp: each lane's
+        // arrival is triggered by the completion of its own copies
+        // (cp.async.mbarrier.arrive.noinc).  The MMA thread orders the
+        // copies' generic-proxy writes before the tensor core's reads with a
+        // proxy fence after its wait.
+        auto publish_copies = [&](uint32_t mbar) { cp_async_arrive_noinc(mbar); };
         uint32_t g = 0;
         int k = 0;
         bool ok = true;
@@ -317,7 +360,7 @@ __global__ void __launch_bounds__(kPersistThreads, 2)
                 }
             } else {
                 warp_load_rows<kRows>(sq, a.q + seq_off, a.tok_stride, it.q0, it.len, lane);
-                cp_async_arrive_noinc(q_full(qb));
+                publish_copies(q_full(qb));
             }
             for (int t = 0; t < it.nt; ++t, ++g) {
                 const int s = static_cast<int>(g % S);
@@ -338,11 +381,11 @@ __global__ void __launch_bounds__(kPersistThreads, 2)
                 } else {
                     warp_load_rows<kTileN>(sk, a.k + seq_off, a.tok_stride, r0, it.len, lane);
                     warp_load_rows<kTileN>(sk + kKVTileBytes, a.v + seq_off, a.tok_stride, r0, it.len, lane);
-                    cp_async_arrive_noinc(kv_full(s));
+                    publish_copies(kv_full(s));
                 }
             }
         }
-        cp_async_wait<0>();
+        cp_async_wait_all();
         if (*fail_flag) {
             // Let the TMA loads still in flight land before the CTA can exit:
             // the newest tile of each ring stage and the newest Q loads.
@@ -356,7 +399,7 @@ __global__ void __launch_bounds__(kPersistThreads, 2)
             const uint32_t idesc_pv = make_idesc(Cvt<T>::kFormat, 1, 64);
             // P V of tile x (the first of its item when `first`, item index kk).
             auto issue_pv = [&](uint32_t x, bool first, int kk) {
-                if (!mbar_wait(p_full(x & 1), (x >> 1) & 1)) return false;
+                if (!mbar_wait(p_full(x & 3), (x >> 2) & 1)) return false;
                 if (first && kk >= 1 && !mbar_wait(o_empty, (kk - 1) & 1)) return false;
                 fence_after_sync();
                 const uint32_t p_addr = tmem + kStreamPCol + (kParts == 2 ? 0u : (x & 1) * 32u);
@@ -371,40 +414,42 @@ __global__ void __launch_bounds__(kPersistThreads, 2)
                 mma_commit(kv_empty(x % S));
                 return true;
             };
-            uint32_t g = 0;
-            int k = 0;
-            bool ok = true;
-            for (int j = blockIdx.x; ok && j < total; j += gridDim.x, ++k) {
-                const Item it = decode_item(j, s_cu, s_ip, a.B, a.H);
-                const int qb = k & 1;
-                if (!mbar_wait(q_full(qb), (k >> 1) & 1)) {
-                    ok = false;
-                    break;
-                }
+            // Two walks over this CTA's tiles: Q K^T runs two tiles ahead of
+            // P V.  P V(g) is issued as soon as P(g) is in TMEM, then Q K^T of
+            // tile g + 2 into the S buffer that the softmax of tile g has
+            // released; the scores of tile g + 1 are already there, so the
+            // softmax never waits for this pair.
+            Walk wq(blockIdx.x, total, s_cu, s_ip, a.B, a.H);
+            Walk wp = wq;
+            uint32_t gq = 0;
+            auto issue_qk = [&]() {
+                const int qb = wq.k & 1;
+                if (wq.t == 0 && !mbar_wait(q_full(qb), (wq.k >> 1) & 1)) return false;
+                if (gq >= 2 && !mbar_wait(s_free(gq & 1), ((gq - 2) >> 1) & 1)) return false;
+                const int s = static_cast<int>(gq % S);
+                if (!mbar_wait(kv_full(s), (gq / S) & 1)) return false;
+                // Tiles filled by cp.async were written through the generic
+                // proxy; order them before the tensor core's reads.
+                fence_async_smem();
+                fence_after_sync();
+                const uint32_t d = tmem + (gq & 1) * static_cast<uint32_t>(kTileN);
                 const uint32_t sq = sQ + qb * kQBytes;
-                for (int t = 0; t < it.nt; ++t, ++g) {
-                    const int s = static_cast<int>(g % S);
-                    if (!mbar_wait(kv_full(s), (g / S) & 1)) {
-                        ok = false;
-                        break;
-                    }
-                    // Tiles filled by cp.async were written through the generic
-                    // proxy; order them before the tensor core's reads.
-                    fence_async_smem();
-                    fence_after_sync();
-                    const uint32_t d = tmem + (g & 1) * static_cast<uint32_t>(kTileN);
-                    const uint32_t sk = sRing + s * 2 * kKVTileBytes;
+                const uint32_t sk = sRing + s * 2 * kKVTileBytes;
 #pragma unroll
-                    for (int ks = 0; ks < 4; ++ks)
-                        mma_f16(d, make_sdesc(sq + ks * 32), make_sdesc(sk + ks * 32), idesc_qk, ks > 0);
-                    mma_commit(s_full(g & 1));
-                    if (t == it.nt - 1) mma_commit(q_empty(qb));
-                    if (t >= 1 && !issue_pv(g - 1, t == 1, k)) {
-                        ok = false;
-                        break;
-                    }
-                }
-                if (ok && !issue_pv(g - 1, it.nt == 1, k)) ok = false;
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_f16(d, make_sdesc(sq + ks * 32), make_sdesc(sk + ks * 32), idesc_qk, ks > 0);
+                mma_commit(s_full(gq & 1));
+                if (wq.t == wq.it.nt - 1) mma_commit(q_empty(qb));
+                ++gq;
+                wq.next();
+                return true;
+            };
+            bool ok = true;
+            for (int i = 0; ok && i < 2 && wq.valid; ++i) ok = issue_qk();
+            for (uint32_t gp = 0; ok && wp.valid; ++gp) {
+                if (!issue_pv(gp, wp.t == 0, wp.k)) ok = false;
+                else if (wq.valid && !issue_qk()) ok = false;
+                wp.next();
             }
             if (!ok) atomicExch(&s_fail, 1);
             // Every MMA this thread issued has completed before TMEM is freed.
@@ -415,11 +460,18 @@ __global__ void __launch_bounds__(kPersistThreads, 2)
         // ---------------- softmax and epilogue (one thread per query row) ----------------
         const uint32_t t_lane = tmem + (static_cast<uint32_t>(warp * 32) << 16);
         constexpr int kPLag = kParts == 2 ? 1 : 2;   // P slots: bf16 one (hi + lo), f16 two
+        // Every product up to tile x has finished.  The phases of each pv_done
+        // barrier are waited for one by one, in order: a parity wait is only
+        // exact while the barrier is at most one phase behind the target, and
+        // warps without rows in a query tile skip the per-tile waits.
         int pv_seen = -1;
         auto confirm_pv = [&](int x) {
-            if (x > pv_seen) {
-                if (!mbar_wait(pv_done(x & 1), (x >> 1) & 1)) atomicExch(&s_fail, 1);
-                pv_seen = x;
+            while (pv_seen < x) {
+                ++pv_seen;
+                if (!mbar_wait(pv_done(pv_seen & 1), (pv_seen >> 1) & 1)) {
+                    atomicExch(&s_fail, 1);
+                    pv_seen = x;
+                }
             }
         };
         const uint64_t sl2 = f2(a.scale_log2, a.scale_log2);
@@ -440,9 +492,12 @@ __global__ void __launch_bounds__(kPersistThreads, 2)
                     break;
                 }
                 fence_after_sync();
+                float sv[64];
+                if (warp_rows) tmem_ld64(t_lane + static_cast<uint32_t>((g & 1) * kTileN), sv);
+                // S(g) is in registers: its TMEM buffer may take Q K^T of tile g + 2.
+                fence_before_sync();
+                mbar_arrive(s_free(g & 1));
                 if (warp_rows) {
-                    float sv[64];
-                    tmem_ld64(t_lane + static_cast<uint32_t>((g & 1) * kTileN), sv);
                     const int valid = min(kTileN, it.len - t * kTileN);
                     if (valid < kTileN) {
 #pragma unroll
@@ -484,8 +539,12 @@ __global__ void __launch_bounds__(kPersistThreads, 2)
                             tmem_st16(t_lane + kStreamOCol + q * 16, part);
                         }
                     }
-                    // The P slot is free once the product that last read it is done.
-                    if (g >= kPLag) confirm_pv(g - kPLag);
+                }
+                // The P slot is free once the product that last read it is done.
+                // Every warp waits here, rows or not, so that each pv_done phase
+                // is waited for while it is the barrier's next one.
+                if (g >= kPLag) confirm_pv(g - kPLag);
+                if (warp_rows) {
                     fence_after_sync();
                     const uint32_t p_col =
                         t_lane + kStreamPCol + (kParts == 2 ? 0u : static_cast<uint32_t>((g & 1) * 32));
@@ -520,7 +579,7 @@ __global__ void __launch_bounds__(kPersistThreads, 2)
                     tmem_wait_st();
                 }
                 fence_before_sync();
-                mbar_arrive(p_full(g & 1));
+                mbar_arrive(p_full(g & 3));
             }
             if (!ok || *fail_flag) break;
 
