@@ -23,7 +23,9 @@
 //              (the last rows of a sequence) by cp.async with zero fill, each
 //              lane's arrival triggered by the completion of its copies
 //              (cp.async.mbarrier.arrive.noinc).  Q is double-buffered, K/V
-//              flow through a 4-stage ring.
+//              flow through a 4-stage ring; the stage of an item's last tile
+//              is handed back by the softmax warps once the epilogue has used
+//              it to stage O for row-contiguous stores.
 //   warp 4     one thread issues every tcgen05.mma.  Q K^T runs two tiles
 //              ahead of P V: P V(g) as soon as P(g) is in TMEM, then S of tile
 //              g + 2 into TMEM buffer g & 1, which the softmax has read S(g)
@@ -234,8 +236,8 @@ __global__ void __launch_bounds__(kPersistThreads, 2)
                              const __grid_constant__ CUtensorMap tm_v, const PersistArgs a) {
     extern __shared__ uint8_t smem_raw[];
     // kv_full[S], kv_empty[S], q_full[2], q_empty[2], s_full[2], p_full[0..1], pv_done[2], o_empty, drain,
-    // s_free[2], p_full[2..3]
-    __shared__ __align__(8) uint64_t s_bar[2 * kPersistStages + 16];
+    // s_free[2], p_full[2..3], o_staged, o_stored
+    __shared__ __align__(8) uint64_t s_bar[2 * kPersistStages + 18];
     __shared__ uint32_t s_tmem;
     __shared__ int s_fail;
 
@@ -265,6 +267,10 @@ __global__ void __launch_bounds__(kPersistThreads, 2)
     const uint32_t o_empty = bar0 + 8u * (2 * S + 10);
     const uint32_t drain = bar0 + 8u * (2 * S + 11);
     auto s_free = [&](int i) { return bar0 + 8u * (2 * S + 12 + i); };
+    // The epilogue's O tile is staged in shared memory / has been stored
+    // (128 arrivals each, one phase per item).
+    const uint32_t o_staged = bar0 + 8u * (2 * S + 16);
+    const uint32_t o_stored = bar0 + 8u * (2 * S + 17);
     volatile int* fail_flag = &s_fail;
 
     // ---- setup: cu_seqlens, barriers, TMEM, item offsets ----
@@ -284,6 +290,8 @@ __global__ void __launch_bounds__(kPersistThreads, 2)
             mbar_init(s_free(i), kSoftmaxThreads);
         }
         mbar_init(o_empty, kSoftmaxThreads);
+        mbar_init(o_staged, kSoftmaxThreads);
+        mbar_init(o_stored, kSoftmaxThreads);
         mbar_init(drain, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         s_fail = 0;
@@ -398,7 +406,9 @@ __global__ void __launch_bounds__(kPersistThreads, 2)
             const uint32_t idesc_qk = make_idesc(Cvt<T>::kFormat, 0, kTileN);
             const uint32_t idesc_pv = make_idesc(Cvt<T>::kFormat, 1, 64);
             // P V of tile x (the first of its item when `first`, item index kk).
-            auto issue_pv = [&](uint32_t x, bool first, int kk) {
+            // The stage of an item's last tile is released by the epilogue,
+            // which stages O there.
+            auto issue_pv = [&](uint32_t x, bool first, bool last, int kk) {
                 if (!mbar_wait(p_full(x & 3), (x >> 2) & 1)) return false;
                 if (first && kk >= 1 && !mbar_wait(o_empty, (kk - 1) & 1)) return false;
                 fence_after_sync();
@@ -411,7 +421,7 @@ __global__ void __launch_bounds__(kPersistThreads, 2)
                         mma_f16_ts(tmem + kStreamOCol, p_addr + part * 32 + ks * 8, make_sdesc(sv + ks * 2048),
                                    idesc_pv, (first && part == 0 && ks == 0) ? 0u : 1u);
                 mma_commit(pv_done(x & 1));
-                mma_commit(kv_empty(x % S));
+                if (!last) mma_commit(kv_empty(x % S));
                 return true;
             };
             // Two walks over this CTA's tiles: Q K^T runs two tiles ahead of
@@ -447,7 +457,7 @@ __global__ void __launch_bounds__(kPersistThreads, 2)
             bool ok = true;
             for (int i = 0; ok && i < 2 && wq.valid; ++i) ok = issue_qk();
             for (uint32_t gp = 0; ok && wp.valid; ++gp) {
-                if (!issue_pv(gp, wp.t == 0, wp.k)) ok = false;
+                if (!issue_pv(gp, wp.t == 0, wp.t == wp.it.nt - 1, wp.k)) ok = false;
                 else if (wq.valid && !issue_qk()) ok = false;
                 wp.next();
             }
@@ -583,19 +593,21 @@ __global__ void __launch_bounds__(kPersistThreads, 2)
             }
             if (!ok || *fail_flag) break;
 
-            // Epilogue: the item's last product, O read out (32 columns at a
-            // time) and stored as O / l, then O released to the next item.
+            // Epilogue.  Once the item's last product is done, the K/V stage of
+            // its last tile is no longer read by anything (its release to the
+            // load warp is left to this epilogue), so O / l is staged there:
+            // each thread writes its row (swizzled 16-byte chunks), O is
+            // released to the next item, and the four warps store the tile
+            // row-contiguously, four 128-byte rows per instruction, instead of
+            // 32 scattered 16-byte pieces.
             confirm_pv(g - 1);
             fence_after_sync();
+            fence_async_smem();
+            const int last_stage = (g - 1) % S;
+            uint8_t* stage = smem_raw + (sRing - raw) + last_stage * 2 * kKVTileBytes;
             if (warp_rows) {
-                const bool store = row < it.len;
                 const float inv = 1.f / (l0 + l1);
                 const uint64_t inv2 = f2(inv, inv);
-                uint4* dst = reinterpret_cast<uint4*>(a.out + static_cast<int64_t>(it.start + row) * a.out_tok_stride +
-                                                      it.h * 64);
-                uint4* cd = (row == 0 && a.cls_out != nullptr)
-                                ? reinterpret_cast<uint4*>(a.cls_out + (static_cast<int64_t>(it.b) * a.H + it.h) * 64)
-                                : nullptr;
 #pragma unroll
                 for (int hf = 0; hf < 2; ++hf) {
                     float ov[32];
@@ -607,18 +619,43 @@ __global__ void __launch_bounds__(kPersistThreads, 2)
                         f2_split(f2_mul(f2(ov[2 * i], ov[2 * i + 1]), inv2), o0, o1);
                         w[i] = Cvt<T>::pack(o0, o1);
                     }
-                    if (store) {
 #pragma unroll
-                        for (int c = 0; c < 4; ++c) {
-                            const uint4 val = make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
-                            dst[hf * 4 + c] = val;
-                            if (cd != nullptr) cd[hf * 4 + c] = val;
-                        }
-                    }
+                    for (int c = 0; c < 4; ++c)
+                        *reinterpret_cast<uint4*>(stage + swz(tid, hf * 4 + c)) =
+                            make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
                 }
             }
             fence_before_sync();
             mbar_arrive(o_empty);
+            mbar_arrive(o_staged);
+            if (!mbar_wait(o_staged, k & 1)) {
+                atomicExch(&s_fail, 1);
+                break;
+            }
+            {
+                const int rows = min(kRows, it.len - it.q0);
+                const int c = lane & 7;
+                uint16_t* cls = a.cls_out != nullptr && it.q0 == 0
+                                    ? a.cls_out + (static_cast<int64_t>(it.b) * a.H + it.h) * 64
+                                    : nullptr;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int r = i * 16 + warp * 4 + (lane >> 3);
+                    if (r < rows) {
+                        const uint4 val = *reinterpret_cast<const uint4*>(stage + swz(r, c));
+                        *reinterpret_cast<uint4*>(a.out + static_cast<int64_t>(it.start + it.q0 + r) * a.out_tok_stride +
+                                                  it.h * 64 + c * 8) = val;
+                        if (r == 0 && cls != nullptr) *reinterpret_cast<uint4*>(cls + c * 8) = val;
+                    }
+                }
+            }
+            // The stage goes back to the load warp once every read of it is done.
+            fence_async_smem();
+            mbar_arrive(o_stored);
+            if (tid == 0) {
+                if (mbar_wait(o_stored, k & 1)) mbar_arrive(kv_empty(last_stage));
+                else atomicExch(&s_fail, 1);
+            }
         }
     }
 
