@@ -145,7 +145,9 @@ RAGGED_API ragged_status ragged_attn_fwd(const void *q, const void *k, const voi
 /* Attention kernels (ragged_set_attn_kernel). */
 #define RAGGED_ATTN_AUTO 0       /* per launch shape (default): RESIDENT for launches too
                                     small to fill the GPU or single-tile sequences,
-                                    PERSISTENT for long sequences, STREAMING otherwise    */
+                                    PERSISTENT for launches of at least 8 (sequence,
+                                    128-query tile, head) items per SM (B <= 1024),
+                                    TCGEN05 for other long sequences, STREAMING otherwise */
 #define RAGGED_ATTN_STREAMING 1  /* mma.sync, K/V tiles streamed, any max_seqlen            */
 #define RAGGED_ATTN_RESIDENT 2   /* mma.sync, whole sequence in shared memory, <= 640 keys */
 #define RAGGED_ATTN_TCGEN05 3    /* tcgen05.mma with TMEM accumulators, K/V streamed, one

@@ -412,12 +412,17 @@ ragged_status ragged_attn_fwd(const void* q, const void* k, const void* v, int64
     }
     // Kernel choice.  AUTO: whole-sequence residency pays off in the
     // latency-bound regime (few CTAs: keys split across warps) and for
-    // single-tile sequences; other launches stream K/V tiles.
+    // single-tile sequences; launches with at least eight (sequence, query
+    // tile, head) items per SM go to the persistent tcgen05 kernel, whose
+    // per-CTA set-up is paid once; the rest stream K/V tiles.
     const int res_tiles = static_cast<int>((max_seqlen + 63) / 64);
+    const int64_t q_tiles = (max_seqlen + 127) / 128;
     int kernel_choice = g_attn_kernel.load(std::memory_order_relaxed);
     if (kernel_choice == RAGGED_ATTN_AUTO) {
         if (max_seqlen <= ragged::resident::kMaxKeys && (res_tiles == 1 || resident_ksplit(B, H, res_tiles) > 1))
             kernel_choice = RAGGED_ATTN_RESIDENT;
+        else if (B <= ragged::tc05::kPersistMaxB && B * H * q_tiles >= 8LL * sm_count())
+            kernel_choice = RAGGED_ATTN_PERSISTENT;
         else if (res_tiles > 4)
             kernel_choice = RAGGED_ATTN_TCGEN05;   // long sequences: many key tiles per query tile
         else

@@ -103,7 +103,7 @@ def test_streaming_kernel_under_a_loose_bound(dtype):
 @pytest.mark.parametrize("kernel", ["auto", "streaming"])
 def test_long_sequences_above_the_resident_limit(dtype, kernel):
     """L_full above the resident limit (640 keys): the streaming kernel, and
-    AUTO (which picks tcgen05 for sequences over 256 keys)."""
+    AUTO (which picks a tcgen05 kernel for sequences over 256 keys)."""
     w = synthetic.make_workload("long", 4, 1000, 2, [1000, 700, 641, 65], dtype, 81)
     check_against_oracle(w, kernel=kernel)
 
