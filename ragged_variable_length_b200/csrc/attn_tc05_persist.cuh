@@ -11,10 +11,11 @@
 // Each CTA copies cu_seqlens into shared memory once, forms the exclusive
 // prefix of H * ceil(L_b / 128) over the sequences, and takes items
 // blockIdx.x, blockIdx.x + gridDim.x, ...; two CTAs share an SM.  TMEM
-// (256 columns: S of two tiles, P, O) and the mbarriers are set up once per
-// CTA, so the per-launch fixed costs of a CTA (cu_seqlens read, TMEM
-// allocation, first loads) are paid once, and the loads of the next item run
-// under the softmax of the current one.
+// (256 columns: S of two tiles, each overwritten in place by its P, and two
+// O buffers for alternate items) and the mbarriers are set up once per CTA,
+// so the per-launch fixed costs of a CTA (cu_seqlens read, TMEM allocation,
+// first loads) are paid once, and the loads of the next item run under the
+// softmax of the current one.
 //
 // Warp roles; they hand off through mbarriers only:
 //   warp 5     loads.  Full tiles by TMA from 3-D tensor maps over
@@ -28,17 +29,17 @@
 //              it to stage O for row-contiguous stores.
 //   warp 4     one thread issues every tcgen05.mma.  Q K^T runs two tiles
 //              ahead of P V: P V(g) as soon as P(g) is in TMEM, then S of tile
-//              g + 2 into TMEM buffer g & 1, which the softmax has read S(g)
-//              out of.  Across items the walks simply continue, so the next
-//              item's first scores are ready when the current item's
-//              epilogue ends.
+//              g + 2 into TMEM buffer g & 1 (in order behind P V(g), which
+//              read P(g) from it).  Across items the walks simply continue.
 //   warps 0-3  softmax, one thread per query row (TMEM lane = row), single
 //              pass with a reference maximum that is raised (and the running
 //              sum and O rescaled) only when a tile exceeds it by more than
-//              2^8; P goes to TMEM (bf16: hi and lo parts).  The pairwise
-//              fp32 work uses the packed f32x2 instructions of sm_100.  The
-//              epilogue reads O from TMEM, releases it to the next item, and
-//              stores O / l (and the CLS row).
+//              2^8; P (bf16: hi and lo parts) replaces S in its TMEM buffer.
+//              The pairwise fp32 work uses the packed f32x2 instructions of
+//              sm_100.  An item's epilogue (O / l and the CLS row) runs after
+//              the first tile of the next item, from the item's own O buffer,
+//              so the softmax warps never wait at an item boundary for the
+//              last product.
 // The tile counter g runs across items, so every buffer parity carries over
 // from one item to the next.
 //
@@ -56,6 +57,10 @@ namespace tc05 {
 
 constexpr int kPersistThreads = 192;
 constexpr int kPersistStages = 4;
+// TMEM per CTA (256 columns): S of two tiles at [0, 64) and [64, 128), each
+// overwritten in place by its P (16-bit pairs; bf16 as hi + lo halves), and
+// two O buffers at [128, 192) and [192, 256), one per alternate item.
+constexpr uint32_t kOBufCol = 128;
 constexpr int kPersistMaxB = 1024;   // cu_seqlens and item offsets live in shared memory
 constexpr int kMmaWarp = 4;
 constexpr int kLoadWarp = 5;
@@ -235,8 +240,8 @@ __global__ void __launch_bounds__(kPersistThreads, 2)
     attn_tc05_persist_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                              const __grid_constant__ CUtensorMap tm_v, const PersistArgs a) {
     extern __shared__ uint8_t smem_raw[];
-    // kv_full[S], kv_empty[S], q_full[2], q_empty[2], s_full[2], p_full[0..1], pv_done[2], o_empty, drain,
-    // s_free[2], p_full[2..3], o_staged, o_stored
+    // kv_full[S], kv_empty[S], q_full[2], q_empty[2], s_full[2], p_full[0..1], pv_done[2], o_empty[0], drain,
+    // o_empty[1], (unused), p_full[2..3], o_staged, o_stored
     __shared__ __align__(8) uint64_t s_bar[2 * kPersistStages + 18];
     __shared__ uint32_t s_tmem;
     __shared__ int s_fail;
@@ -264,9 +269,9 @@ __global__ void __launch_bounds__(kPersistThreads, 2)
     // waits until every warp has read S(g + 1)).
     auto p_full = [&](int i) { return bar0 + 8u * (i < 2 ? 2 * S + 6 + i : 2 * S + 14 + (i - 2)); };
     auto pv_done = [&](int i) { return bar0 + 8u * (2 * S + 8 + i); };
-    const uint32_t o_empty = bar0 + 8u * (2 * S + 10);
+    // O buffer i has been read out by the epilogue of its item.
+    auto o_empty = [&](int i) { return bar0 + 8u * (i == 0 ? 2 * S + 10 : 2 * S + 12); };
     const uint32_t drain = bar0 + 8u * (2 * S + 11);
-    auto s_free = [&](int i) { return bar0 + 8u * (2 * S + 12 + i); };
     // The epilogue's O tile is staged in shared memory / has been stored
     // (128 arrivals each, one phase per item).
     const uint32_t o_staged = bar0 + 8u * (2 * S + 16);
@@ -287,9 +292,8 @@ __global__ void __launch_bounds__(kPersistThreads, 2)
             mbar_init(p_full(i), kSoftmaxThreads);
             mbar_init(p_full(i + 2), kSoftmaxThreads);
             mbar_init(pv_done(i), 1);
-            mbar_init(s_free(i), kSoftmaxThreads);
+            mbar_init(o_empty(i), kSoftmaxThreads);
         }
-        mbar_init(o_empty, kSoftmaxThreads);
         mbar_init(o_staged, kSoftmaxThreads);
         mbar_init(o_stored, kSoftmaxThreads);
         mbar_init(drain, 1);
@@ -408,17 +412,21 @@ __global__ void __launch_bounds__(kPersistThreads, 2)
             // P V of tile x (the first of its item when `first`, item index kk).
             // The stage of an item's last tile is released by the epilogue,
             // which stages O there.
+            // P V of tile x of item kk: P sits in S buffer x & 1, O in buffer
+            // kk & 1.  An item's first product overwrites its O buffer, which
+            // the epilogue of item kk - 2 must have read out.
             auto issue_pv = [&](uint32_t x, bool first, bool last, int kk) {
                 if (!mbar_wait(p_full(x & 3), (x >> 2) & 1)) return false;
-                if (first && kk >= 1 && !mbar_wait(o_empty, (kk - 1) & 1)) return false;
+                if (first && kk >= 2 && !mbar_wait(o_empty(kk & 1), ((kk >> 1) - 1) & 1)) return false;
                 fence_after_sync();
-                const uint32_t p_addr = tmem + kStreamPCol + (kParts == 2 ? 0u : (x & 1) * 32u);
+                const uint32_t p_addr = tmem + (x & 1) * static_cast<uint32_t>(kTileN);
+                const uint32_t o_addr = tmem + kOBufCol + (kk & 1) * 64u;
                 const uint32_t sv = sRing + (x % S) * 2 * kKVTileBytes + kKVTileBytes;
 #pragma unroll
                 for (int part = 0; part < kParts; ++part)
 #pragma unroll
                     for (int ks = 0; ks < 4; ++ks)
-                        mma_f16_ts(tmem + kStreamOCol, p_addr + part * 32 + ks * 8, make_sdesc(sv + ks * 2048),
+                        mma_f16_ts(o_addr, p_addr + part * 32 + ks * 8, make_sdesc(sv + ks * 2048),
                                    idesc_pv, (first && part == 0 && ks == 0) ? 0u : 1u);
                 mma_commit(pv_done(x & 1));
                 if (!last) mma_commit(kv_empty(x % S));
@@ -426,16 +434,16 @@ __global__ void __launch_bounds__(kPersistThreads, 2)
             };
             // Two walks over this CTA's tiles: Q K^T runs two tiles ahead of
             // P V.  P V(g) is issued as soon as P(g) is in TMEM, then Q K^T of
-            // tile g + 2 into the S buffer that the softmax of tile g has
-            // released; the scores of tile g + 1 are already there, so the
-            // softmax never waits for this pair.
+            // tile g + 2 into S buffer g & 1: the tensor core executes one
+            // thread's MMAs in order, so P V(g) has read P(g) out of that
+            // buffer before the new scores land in it.  The scores of tile
+            // g + 1 are already there, so the softmax never waits for them.
             Walk wq(blockIdx.x, total, s_cu, s_ip, a.B, a.H);
             Walk wp = wq;
             uint32_t gq = 0;
             auto issue_qk = [&]() {
                 const int qb = wq.k & 1;
                 if (wq.t == 0 && !mbar_wait(q_full(qb), (wq.k >> 1) & 1)) return false;
-                if (gq >= 2 && !mbar_wait(s_free(gq & 1), ((gq - 2) >> 1) & 1)) return false;
                 const int s = static_cast<int>(gq % S);
                 if (!mbar_wait(kv_full(s), (gq / S) & 1)) return false;
                 // Tiles filled by cp.async were written through the generic
@@ -469,11 +477,9 @@ __global__ void __launch_bounds__(kPersistThreads, 2)
     } else {
         // ---------------- softmax and epilogue (one thread per query row) ----------------
         const uint32_t t_lane = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-        constexpr int kPLag = kParts == 2 ? 1 : 2;   // P slots: bf16 one (hi + lo), f16 two
         // Every product up to tile x has finished.  The phases of each pv_done
         // barrier are waited for one by one, in order: a parity wait is only
-        // exact while the barrier is at most one phase behind the target, and
-        // warps without rows in a query tile skip the per-tile waits.
+        // exact while the barrier is at most one phase behind the target.
         int pv_seen = -1;
         auto confirm_pv = [&](int x) {
             while (pv_seen < x) {
@@ -484,17 +490,87 @@ __global__ void __launch_bounds__(kPersistThreads, 2)
                 }
             }
         };
+        // Epilogue of item kk (its last tile gl, running sum lsum): once the
+        // item's last product is done, the K/V stage of tile gl is no longer
+        // read by anything (its release to the load warp is left to this
+        // epilogue), so O / l is staged there: each thread writes its row
+        // (swizzled 16-byte chunks), O buffer kk & 1 is released, and the four
+        // warps store the tile four 128-byte rows per instruction.
+        auto epilogue = [&](const Item& it, int kk, int gl, float lsum) {
+            confirm_pv(gl);
+            fence_after_sync();
+            fence_async_smem();
+            const int last_stage = gl % S;
+            uint8_t* stage = smem_raw + (sRing - raw) + last_stage * 2 * kKVTileBytes;
+            if (it.q0 + warp * 32 < it.len) {
+                const float inv = 1.f / lsum;
+                const uint64_t inv2 = f2(inv, inv);
+                const uint32_t o_addr = t_lane + kOBufCol + (kk & 1) * 64u;
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf) {
+                    float ov[32];
+                    tmem_ld32(o_addr + hf * 32, ov);
+                    uint32_t w[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        float o0, o1;
+                        f2_split(f2_mul(f2(ov[2 * i], ov[2 * i + 1]), inv2), o0, o1);
+                        w[i] = Cvt<T>::pack(o0, o1);
+                    }
+#pragma unroll
+                    for (int c = 0; c < 4; ++c)
+                        *reinterpret_cast<uint4*>(stage + swz(tid, hf * 4 + c)) =
+                            make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+                }
+            }
+            fence_before_sync();
+            mbar_arrive(o_empty(kk & 1));
+            mbar_arrive(o_staged);
+            if (!mbar_wait(o_staged, kk & 1)) {
+                atomicExch(&s_fail, 1);
+                return false;
+            }
+            const int rows = min(kRows, it.len - it.q0);
+            const int c = lane & 7;
+            uint16_t* cls = a.cls_out != nullptr && it.q0 == 0
+                                ? a.cls_out + (static_cast<int64_t>(it.b) * a.H + it.h) * 64
+                                : nullptr;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int r = i * 16 + warp * 4 + (lane >> 3);
+                if (r < rows) {
+                    const uint4 val = *reinterpret_cast<const uint4*>(stage + swz(r, c));
+                    *reinterpret_cast<uint4*>(a.out + static_cast<int64_t>(it.start + it.q0 + r) * a.out_tok_stride +
+                                              it.h * 64 + c * 8) = val;
+                    if (r == 0 && cls != nullptr) *reinterpret_cast<uint4*>(cls + c * 8) = val;
+                }
+            }
+            // The stage goes back to the load warp once every read of it is done.
+            fence_async_smem();
+            mbar_arrive(o_stored);
+            if (tid == 0) {
+                if (mbar_wait(o_stored, kk & 1)) mbar_arrive(kv_empty(last_stage));
+                else atomicExch(&s_fail, 1);
+            }
+            return true;
+        };
         const uint64_t sl2 = f2(a.scale_log2, a.scale_log2);
+        // The epilogue of an item runs after the first tile of the next one,
+        // by when its last product has long finished.
+        bool pending = false;
+        Item p_it{};
+        int p_k = 0, p_gl = 0;
+        float p_l = 0.f;
         int g = 0;
         int k = 0;
-        for (int j = blockIdx.x; j < total; j += gridDim.x, ++k) {
+        bool ok = true;
+        for (int j = blockIdx.x; ok && j < total; j += gridDim.x, ++k) {
             if (*fail_flag) break;
             const Item it = decode_item(j, s_cu, s_ip, a.B, a.H);
-            const int row = it.q0 + tid;
             const bool warp_rows = it.q0 + warp * 32 < it.len;
+            const uint32_t o_buf = t_lane + kOBufCol + (k & 1) * 64u;
             float m_ref = -INFINITY;   // reference maximum (log2 units) of this row
             float l0 = 0.f, l1 = 0.f;  // running sum, even / odd keys
-            bool ok = true;
             for (int t = 0; t < it.nt; ++t, ++g) {
                 if (!mbar_wait(s_full(g & 1), (g >> 1) & 1)) {
                     atomicExch(&s_fail, 1);
@@ -502,12 +578,10 @@ __global__ void __launch_bounds__(kPersistThreads, 2)
                     break;
                 }
                 fence_after_sync();
-                float sv[64];
-                if (warp_rows) tmem_ld64(t_lane + static_cast<uint32_t>((g & 1) * kTileN), sv);
-                // S(g) is in registers: its TMEM buffer may take Q K^T of tile g + 2.
-                fence_before_sync();
-                mbar_arrive(s_free(g & 1));
+                const uint32_t s_buf = t_lane + static_cast<uint32_t>((g & 1) * kTileN);
                 if (warp_rows) {
+                    float sv[64];
+                    tmem_ld64(s_buf, sv);
                     const int valid = min(kTileN, it.len - t * kTileN);
                     if (valid < kTileN) {
 #pragma unroll
@@ -534,33 +608,26 @@ __global__ void __launch_bounds__(kPersistThreads, 2)
                         m_ref = mt;
                     }
                     if (t > 0 && __any_sync(kFullMask, grow)) {
-                        // O holds the finished products of this item's tiles so far.
+                        // O holds the finished products of this item's tiles so far;
+                        // 16 columns at a time, since sv is still live here.
                         confirm_pv(g - 1);
                         fence_after_sync();
-                        // 16 columns at a time: sv is still live here.
                         const uint64_t a2 = f2(alpha, alpha);
 #pragma unroll
                         for (int q = 0; q < 4; ++q) {
                             float part[16];
-                            tmem_ld16(t_lane + kStreamOCol + q * 16, part);
+                            tmem_ld16(o_buf + q * 16, part);
 #pragma unroll
                             for (int i = 0; i < 8; ++i)
                                 f2_split(f2_mul(f2(part[2 * i], part[2 * i + 1]), a2), part[2 * i], part[2 * i + 1]);
-                            tmem_st16(t_lane + kStreamOCol + q * 16, part);
+                            tmem_st16(o_buf + q * 16, part);
                         }
                     }
-                }
-                // The P slot is free once the product that last read it is done.
-                // Every warp waits here, rows or not, so that each pv_done phase
-                // is waited for while it is the barrier's next one.
-                if (g >= kPLag) confirm_pv(g - kPLag);
-                if (warp_rows) {
-                    fence_after_sync();
-                    const uint32_t p_col =
-                        t_lane + kStreamPCol + (kParts == 2 ? 0u : static_cast<uint32_t>((g & 1) * 32));
+                    // P(g) replaces S(g) in its TMEM buffer: the product that
+                    // read the buffer's previous P was issued, and so executed,
+                    // before the scores that have just been read.
                     const uint64_t nm = f2(-m_ref, -m_ref);
                     uint64_t lsum = f2(l0, l1);
-                    // Two halves of 32 keys, each stored as soon as it is ready.
 #pragma unroll
                     for (int hf = 0; hf < 2; ++hf) {
                         uint32_t p_hi[16], p_lo[16];
@@ -582,81 +649,35 @@ __global__ void __launch_bounds__(kPersistThreads, 2)
                                 p_lo[i] = Cvt<T>::pack(r0, r1);
                             }
                         }
-                        tmem_st16_u(p_col + hf * 16, p_hi);
-                        if constexpr (kParts == 2) tmem_st16_u(p_col + 32 + hf * 16, p_lo);
+                        tmem_st16_u(s_buf + hf * 16, p_hi);
+                        if constexpr (kParts == 2) tmem_st16_u(s_buf + 32 + hf * 16, p_lo);
                     }
                     f2_split(lsum, l0, l1);
                     tmem_wait_st();
                 }
+                // Every warp, rows or not, takes each pv_done phase while it is
+                // the barrier's next one (products up to g - 2 are long done).
+                // This comes before the arrival for tile g: after it, P V(g)
+                // may complete and move barrier g & 1 one phase past g - 2.
+                if (g >= 2) confirm_pv(g - 2);
                 fence_before_sync();
                 mbar_arrive(p_full(g & 3));
+                if (t == 0 && pending) {
+                    if (!epilogue(p_it, p_k, p_gl, p_l)) {
+                        ok = false;
+                        break;
+                    }
+                    pending = false;
+                }
             }
             if (!ok || *fail_flag) break;
-
-            // Epilogue.  Once the item's last product is done, the K/V stage of
-            // its last tile is no longer read by anything (its release to the
-            // load warp is left to this epilogue), so O / l is staged there:
-            // each thread writes its row (swizzled 16-byte chunks), O is
-            // released to the next item, and the four warps store the tile
-            // row-contiguously, four 128-byte rows per instruction, instead of
-            // 32 scattered 16-byte pieces.
-            confirm_pv(g - 1);
-            fence_after_sync();
-            fence_async_smem();
-            const int last_stage = (g - 1) % S;
-            uint8_t* stage = smem_raw + (sRing - raw) + last_stage * 2 * kKVTileBytes;
-            if (warp_rows) {
-                const float inv = 1.f / (l0 + l1);
-                const uint64_t inv2 = f2(inv, inv);
-#pragma unroll
-                for (int hf = 0; hf < 2; ++hf) {
-                    float ov[32];
-                    tmem_ld32(t_lane + kStreamOCol + hf * 32, ov);
-                    uint32_t w[16];
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        float o0, o1;
-                        f2_split(f2_mul(f2(ov[2 * i], ov[2 * i + 1]), inv2), o0, o1);
-                        w[i] = Cvt<T>::pack(o0, o1);
-                    }
-#pragma unroll
-                    for (int c = 0; c < 4; ++c)
-                        *reinterpret_cast<uint4*>(stage + swz(tid, hf * 4 + c)) =
-                            make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
-                }
-            }
-            fence_before_sync();
-            mbar_arrive(o_empty);
-            mbar_arrive(o_staged);
-            if (!mbar_wait(o_staged, k & 1)) {
-                atomicExch(&s_fail, 1);
-                break;
-            }
-            {
-                const int rows = min(kRows, it.len - it.q0);
-                const int c = lane & 7;
-                uint16_t* cls = a.cls_out != nullptr && it.q0 == 0
-                                    ? a.cls_out + (static_cast<int64_t>(it.b) * a.H + it.h) * 64
-                                    : nullptr;
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const int r = i * 16 + warp * 4 + (lane >> 3);
-                    if (r < rows) {
-                        const uint4 val = *reinterpret_cast<const uint4*>(stage + swz(r, c));
-                        *reinterpret_cast<uint4*>(a.out + static_cast<int64_t>(it.start + it.q0 + r) * a.out_tok_stride +
-                                                  it.h * 64 + c * 8) = val;
-                        if (r == 0 && cls != nullptr) *reinterpret_cast<uint4*>(cls + c * 8) = val;
-                    }
-                }
-            }
-            // The stage goes back to the load warp once every read of it is done.
-            fence_async_smem();
-            mbar_arrive(o_stored);
-            if (tid == 0) {
-                if (mbar_wait(o_stored, k & 1)) mbar_arrive(kv_empty(last_stage));
-                else atomicExch(&s_fail, 1);
-            }
+            pending = true;
+            p_it = it;
+            p_k = k;
+            p_gl = g - 1;
+            p_l = l0 + l1;
         }
+        if (ok && pending && !*fail_flag) epilogue(p_it, p_k, p_gl, p_l);
     }
 
     fence_before_sync();
