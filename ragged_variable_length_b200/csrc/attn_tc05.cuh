@@ -1,33 +1,16 @@
 // Ragged bidirectional attention on the 5th-generation tensor cores
-// (tcgen05.mma with TMEM accumulators), f16 / bf16, head_dim 64.
+// (tcgen05.mma with TMEM accumulators), f16 / bf16, head_dim 64: the shared
+// tcgen05 / TMEM / mbarrier helpers and the per-tile streaming kernel.
 //
 // Operation ("Dispatch-Aware Ragged Attention for Pruned Vision Transformers",
 // abstract; radpulse section "Bypassing the binding"): per sequence b and head
 // h, O = softmax(scale Q K^T) V over the sequence's own rows.
 //
-// One CTA (4 warps) per (128-query tile, head, sequence), all of the
-// sequence's K and V resident in shared memory (up to 640 keys):
-//   - every load (Q tile, all K/V tiles) is issued at once with cp.async into
-//     128-byte-swizzled tiles, which are the canonical SWIZZLE_128B operand
-//     layouts of tcgen05 (K-major for Q, K and P; MN-major for V);
-//   - thread 0 issues S = Q K^T for each 64-key tile into TMEM as soon as
-//     that tile has landed (M = 128, N = 64, K = 64 in four K = 16 steps);
-//   - the softmax is one thread per query row (TMEM lane = row): the exact row
-//     maximum over all keys first, then p = exp2(s scale log2e - m) and the
-//     row sum, so the output never needs rescaling.  P is written to a
-//     double-buffered shared tile (bf16: split into bf16 hi + lo parts, each
-//     multiplied with V, so the product carries ~16 bits of P);
-//   - thread 0 accumulates O += P V into TMEM (N = 64 dims, K = 64 keys per
-//     tile), tcgen05.commit releasing each P buffer;
-//   - the epilogue reads O from TMEM, divides by the row sum and stores the
-//     row (and the CLS row).
-// S occupies TMEM columns [0, 448) and O columns [448, 512).  Sequences
-// longer than 448 keys take two passes over key chunks of 448: the first for
-// the row maxima, the second recomputes S for the probabilities.
-//
-// Every mbarrier wait is bounded; a wait that gives up sets
-// RAGGED_DEV_TIMEOUT in the status word and the CTA skips to its teardown
-// (TMEM is always freed).
+// Shared-memory operand tiles use the 128-byte XOR swizzle of mma_attn::swz,
+// which is the canonical SWIZZLE_128B layout of tcgen05 (K-major for Q, K and
+// P; MN-major for V; 8-row groups 1024 bytes apart).  Every mbarrier wait is
+// bounded; a wait that gives up sets RAGGED_DEV_TIMEOUT in the status word and
+// the CTA skips to its teardown (TMEM is always freed).
 #pragma once
 
 #include "attn_resident.cuh"
@@ -38,24 +21,11 @@ namespace tc05 {
 using mma_attn::swz;
 using resident::PackedRows;
 
-constexpr int kThreads = 128;
 constexpr int kRows = 128;            // query rows per CTA (MMA M)
 constexpr int kTileN = 64;            // keys per tile
-constexpr int kChunkTiles = 7;        // key tiles per TMEM S chunk (448 columns)
-constexpr int kMaxTiles = 10;         // 640 keys resident
-constexpr int kMaxKeys = kMaxTiles * kTileN;
-constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kOCol = kChunkTiles * kTileN;   // 448
 constexpr int kQBytes = kRows * 128;               // 16 KB
 constexpr int kKVTileBytes = kTileN * 128;         // 8 KB
-constexpr int kPTileBytes = kRows * 128;           // 16 KB (128 rows x 64 keys)
-constexpr int kMaxDynSmem = 230400;                // dynamic part, under the 227 KB per-block limit
 constexpr uint32_t kSpinLimit = 1u << 22;
-
-// Dynamic shared memory: 1 KB alignment slack, Q, K tiles, V tiles, P slots.
-__host__ __device__ constexpr int smem_bytes(int key_tiles, int p_slots, int p_parts) {
-    return 1024 + kQBytes + 2 * key_tiles * kKVTileBytes + p_slots * p_parts * kPTileBytes;
-}
 
 // ---- instruction and shared-memory descriptors -------------------------------
 
@@ -179,233 +149,14 @@ struct Cvt<__nv_bfloat16> {
     }
 };
 
-template <typename T>
-__global__ void __launch_bounds__(kThreads, 1)
-    attn_tc05_kernel(PackedRows src, int key_tiles, int p_slots, float scale_log2, int H,
-                     uint16_t* __restrict__ out, int64_t out_tok_stride, uint16_t* __restrict__ cls_out) {
-    extern __shared__ uint8_t smem_raw[];
-    __shared__ __align__(8) uint64_t s_mbar[4];   // 0: S ready, 1: O ready, 2, 3: P slot free
-    __shared__ uint32_t s_tmem;
-    __shared__ int s_fail;
-
-    const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-    if (!src.begin(b, h, nullptr, nullptr)) return;
-    const int len = src.len, start = src.start;
-    const int q0 = qt * kRows;
-    if (q0 >= len) return;
-    const int nt = (len + kTileN - 1) / kTileN;
-    const int tid = threadIdx.x, warp = tid >> 5;
-    constexpr int kParts = Cvt<T>::kParts;
-
-    const uint32_t raw = smem_addr(smem_raw);
-    const uint32_t sQ = (raw + 1023u) & ~1023u;
-    const uint32_t sK = sQ + kQBytes;
-    const uint32_t sV = sK + key_tiles * kKVTileBytes;
-    const uint32_t sP = sV + key_tiles * kKVTileBytes;
-    const uint32_t slot_bytes = kParts * kPTileBytes;
-    uint8_t* gP = smem_raw + (sP - raw);
-
-    // Loads: group 0 = Q + key tile 0, group t = key tile t.
-    resident::load_tile<kRows>(sQ, src, 0, q0, len);
-    for (int t = 0; t < nt; ++t) {
-        resident::load_tile<kTileN>(sK + t * kKVTileBytes, src, 1, t * kTileN, len);
-        resident::load_tile<kTileN>(sV + t * kKVTileBytes, src, 2, t * kTileN, len);
-        cp_async_commit();
-    }
-
-    const uint32_t mbar0 = smem_addr(&s_mbar[0]);
-    if (tid == 0) {
-        for (int i = 0; i < 4; ++i) mbar_init(mbar0 + 8 * i, 1);
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-        s_fail = 0;
-    }
-    if (warp == 0) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(&s_tmem)),
-                     "r"(kTmemCols)
-                     : "memory");
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-    }
-    fence_before_sync();
-    __syncthreads();
-    fence_after_sync();
-    const uint32_t tmem = s_tmem;
-    const uint32_t t_lane = tmem + (static_cast<uint32_t>(warp * 32) << 16);   // this warp's TMEM lanes
-
-    const uint32_t idesc_qk = make_idesc(Cvt<T>::kFormat, 0, kTileN);
-    const uint32_t idesc_pv = make_idesc(Cvt<T>::kFormat, 1, 64);
-    const int row = q0 + tid;               // this thread's query row (TMEM lane = tid)
-    const int nchunks = (nt + kChunkTiles - 1) / kChunkTiles;
-    uint32_t s_phase = 0;
-    uint32_t p_phase[2] = {0, 0};
-    float m = -INFINITY, l = 0.f;
-
-    // S = Q K^T for the tiles of one chunk, issued tile by tile; when
-    // wait_loads, each tile's cp.async group is awaited first (first pass).
-    auto issue_chunk = [&](int c, bool wait_loads) {
-        const int t0 = c * kChunkTiles, t1 = min(nt, t0 + kChunkTiles);
-        for (int t = t0; t < t1; ++t) {
-            if (wait_loads) {
-                resident::cp_async_wait_pending(nt - 1 - t);
-                fence_async_smem();
-            }
-            fence_before_sync();
-            __syncthreads();
-            if (tid == 0) {
-                fence_after_sync();
-                const uint32_t d = tmem + static_cast<uint32_t>((t - t0) * kTileN);
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    mma_f16(d, make_sdesc(sQ + ks * 32), make_sdesc(sK + t * kKVTileBytes + ks * 32), idesc_qk,
-                            ks > 0);
-            }
-        }
-        if (tid == 0) mma_commit(mbar0);
-        if (!mbar_wait(mbar0, s_phase)) atomicExch(&s_fail, 1);
-        s_phase ^= 1;
-        fence_after_sync();
-    };
-
-    // ---- pass 1: exact row maxima over all keys ----
-    for (int c = 0; c < nchunks; ++c) {
-        if (c > 0) {   // the previous chunk's S must be fully read before it is overwritten
-            fence_before_sync();
-            __syncthreads();
-        }
-        issue_chunk(c, c == 0);
-        if (c == 0 && nchunks > 1) {   // later chunks' loads are awaited here once
-            resident::cp_async_wait_pending(0);
-            fence_async_smem();
-        }
-        const int t0 = c * kChunkTiles, t1 = min(nt, t0 + kChunkTiles);
-        for (int t = t0; t < t1; ++t) {
-#pragma unroll
-            for (int g = 0; g < 4; ++g) {
-                float v[16];
-                tmem_ld16(t_lane + static_cast<uint32_t>((t - t0) * kTileN + g * 16), v);
-#pragma unroll
-                for (int i = 0; i < 16; ++i)
-                    if (t * kTileN + g * 16 + i < len) m = fmaxf(m, v[i]);
-            }
-        }
-    }
-    const float mb = m * scale_log2;
-
-    // ---- pass 2: probabilities, P V ----
-    for (int c = 0; c < nchunks; ++c) {
-        if (nchunks > 1) {
-            fence_before_sync();
-            __syncthreads();
-            issue_chunk(c, false);
-        }
-        if (s_fail) break;
-        const int t0 = c * kChunkTiles, t1 = min(nt, t0 + kChunkTiles);
-        for (int t = t0; t < t1; ++t) {
-            const int slot = p_slots == 2 ? (t & 1) : 0;
-            if (t >= p_slots) {   // the P V product of tile t - p_slots has released this slot
-                if (!mbar_wait(mbar0 + 16 + 8 * slot, p_phase[slot])) atomicExch(&s_fail, 1);
-                p_phase[slot] ^= 1;
-            }
-            uint8_t* p_hi = gP + slot * slot_bytes;
-#pragma unroll
-            for (int g = 0; g < 4; ++g) {
-                float v[16];
-                tmem_ld16(t_lane + static_cast<uint32_t>((t - t0) * kTileN + g * 16), v);
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const bool ok = t * kTileN + g * 16 + i < len;
-                    v[i] = ok ? mma_attn::fast_exp2(fmaf(v[i], scale_log2, -mb)) : 0.f;
-                    l += v[i];
-                }
-#pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    uint32_t w[4];
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) w[i] = Cvt<T>::pack(v[half * 8 + 2 * i], v[half * 8 + 2 * i + 1]);
-                    const int chunk = g * 2 + half;
-                    *reinterpret_cast<uint4*>(p_hi + swz(tid, chunk)) = make_uint4(w[0], w[1], w[2], w[3]);
-                    if constexpr (kParts == 2) {
-                        uint32_t r[4];
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            __nv_bfloat162 hb = *reinterpret_cast<__nv_bfloat162*>(&w[i]);
-                            const float2 f = __bfloat1622float2(hb);
-                            r[i] = Cvt<T>::pack(v[half * 8 + 2 * i] - f.x, v[half * 8 + 2 * i + 1] - f.y);
-                        }
-                        *reinterpret_cast<uint4*>(p_hi + kPTileBytes + swz(tid, chunk)) =
-                            make_uint4(r[0], r[1], r[2], r[3]);
-                    }
-                }
-            }
-            fence_async_smem();
-            fence_before_sync();
-            __syncthreads();
-            if (s_fail) break;
-            if (tid == 0) {
-                fence_after_sync();
-                const uint32_t p_addr = sP + slot * slot_bytes;
-#pragma unroll
-                for (int part = 0; part < kParts; ++part)
-#pragma unroll
-                    for (int ks = 0; ks < 4; ++ks)
-                        mma_f16(tmem + kOCol, make_sdesc(p_addr + part * kPTileBytes + ks * 32),
-                                make_sdesc(sV + t * kKVTileBytes + ks * 2048), idesc_pv,
-                                (t > 0 || part > 0 || ks > 0) ? 1u : 0u);
-                mma_commit(mbar0 + 16 + 8 * slot);
-            }
-        }
-    }
-
-    // ---- epilogue: O / l ----
-    if (tid == 0 && !s_fail) mma_commit(mbar0 + 8);
-    __syncthreads();
-    if (!s_fail) {
-        if (!mbar_wait(mbar0 + 8, 0)) {
-            atomicExch(&s_fail, 1);
-        } else {
-            fence_after_sync();
-            const float inv = 1.f / l;
-            uint32_t w[32];
-#pragma unroll
-            for (int g = 0; g < 4; ++g) {
-                float v[16];
-                tmem_ld16(t_lane + kOCol + g * 16, v);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) w[g * 8 + i] = Cvt<T>::pack(v[2 * i] * inv, v[2 * i + 1] * inv);
-            }
-            if (row < len) {
-                uint4* dst = reinterpret_cast<uint4*>(out + static_cast<int64_t>(start + row) * out_tok_stride +
-                                                      h * 64);
-#pragma unroll
-                for (int c = 0; c < 8; ++c) dst[c] = make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
-                if (row == 0 && cls_out != nullptr) {
-                    uint4* cd = reinterpret_cast<uint4*>(cls_out + (static_cast<int64_t>(b) * H + h) * 64);
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) cd[c] = make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
-                }
-            }
-        }
-    }
-
-    // ---- teardown: loads drained, TMEM freed ----
-    resident::cp_async_wait_pending(0);
-    fence_before_sync();
-    __syncthreads();
-    if (s_fail && tid == 0) raise_status(RAGGED_DEV_TIMEOUT);
-    if (warp == 0) {
-        fence_after_sync();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
-    }
-}
-
-
 // ---------------------------------------------------------------------------
-// Streaming variant: two CTAs per SM.
+// Per-tile streaming kernel: one CTA per (128-query tile, head, sequence),
+// two CTAs per SM.
 //
-// Same operation as attn_tc05_kernel, but the K/V tiles of a sequence flow
-// through a 5-stage shared-memory ring (loads run four tiles ahead), and the
-// probabilities never touch shared memory: each softmax thread stores its
-// row of P into TMEM (16-bit values packed two per column, row = lane) and
-// the P V product reads its A operand from TMEM.  TMEM per CTA (256 columns):
+// The K/V tiles of a sequence flow through a 5-stage shared-memory ring (loads
+// run four tiles ahead), and the probabilities never touch shared memory:
+// each softmax thread stores its row of P into TMEM (16-bit values packed two
+// per column, row = lane) and the P V product reads its A operand from TMEM.  TMEM per CTA (256 columns):
 //   [0, 64) and [64, 128)   S of tiles t (even / odd)
 //   [128, 192)              P: two f16 slots of 32 columns, or the bf16 hi/lo pair
 //   [192, 256)              O

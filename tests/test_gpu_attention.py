@@ -141,7 +141,7 @@ def test_tcgen05_rescale_path(kernel):
 @pytest.mark.parametrize("dtype", ["bf16", "f16"])
 @pytest.mark.parametrize("kernel", list(KERNELS))
 def test_hires_lengths_448_449_576_577_640(dtype, kernel):
-    """Around the tcgen05 kernel's single-pass limit (448 keys) and the resident limit (640)."""
+    """Lengths around whole key tiles (448 = 7 x 64, 576 = 9 x 64), the 577 tokens of a 384x384 ViT, and the resident limit (640)."""
     w = synthetic.make_workload("hires_edges", 6, 640, 2, [577, 576, 300, 640, 448, 449], dtype, 78)
     check_against_oracle(w, kernel=kernel)
 
