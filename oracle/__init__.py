@@ -15,6 +15,9 @@ Vision Transformers"):
                       mask, no KV cache, no padding
   unpack_cls          radpulse "Integrated pack pipeline": extract the CLS token
   unpack              scatter the packed rows back to their dense positions
+  mask_topk / mask_l2 keep-mask producers (radpulse "Integrated pack
+                      pipeline": the pipeline serves any pruning method, e.g.
+                      Threshold-l2); the rules are readings, see the C file
 """
 from __future__ import annotations
 
@@ -66,6 +69,10 @@ def bind(path: str):
     lib.oracle_attention.restype = ctypes.c_int
     lib.oracle_num_cores.argtypes = []
     lib.oracle_num_cores.restype = ctypes.c_int
+    lib.oracle_mask_topk.argtypes = [vp, i64, i64, vp, vp]
+    lib.oracle_mask_topk.restype = None
+    lib.oracle_mask_l2.argtypes = [vp, ctypes.c_int, i64, i64, i64, i64, ctypes.c_double, vp]
+    lib.oracle_mask_l2.restype = None
     return lib
 
 
@@ -196,3 +203,26 @@ def pipeline(w, seqs: Optional[Sequence[int]] = None, threads: int = 0) -> dict:
                     seqs=seqs, threads=threads)
     cls = out[cu[:-1]] if w.B else np.zeros((0, w.H, w.d))
     return {"cu": cu, "src_idx": src, "packed": packed, "out": out, "cls": cls}
+
+
+def mask_topk(scores: np.ndarray, keep_count: np.ndarray) -> np.ndarray:
+    """Top-k keep mask: CLS plus the k_b - 1 highest-scoring other tokens of
+    image b (ties: lower index; NaN ranks last); k_b clamped to [1, L_full]."""
+    scores = np.ascontiguousarray(scores, dtype=np.float32)
+    B, L_full = scores.shape
+    kc = np.ascontiguousarray(keep_count, dtype=np.int32).reshape(B)
+    keep = np.zeros((B, L_full), dtype=np.uint8)
+    _load().oracle_mask_topk(_ptr(scores), B, L_full, _ptr(kc), _ptr(keep))
+    return keep
+
+
+def mask_l2(x: np.ndarray, dtype: str, tau: float) -> np.ndarray:
+    """Threshold-l2 keep mask of x [B, L_full, C] (storage format of dtype):
+    token kept when its Euclidean norm is >= tau; CLS always kept."""
+    x = np.ascontiguousarray(x)
+    if x.dtype != _STORAGE[dtype]:
+        raise ValueError(f"x dtype {x.dtype} does not store {dtype}")
+    B, L_full, C = x.shape
+    keep = np.zeros((B, L_full), dtype=np.uint8)
+    _load().oracle_mask_l2(_ptr(x), DTYPE_CODES[dtype], B, L_full, C, C, float(tau), _ptr(keep))
+    return keep

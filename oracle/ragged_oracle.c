@@ -295,3 +295,87 @@ int oracle_attention(const void *q, const void *k, const void *v, int dtype,
     free(all);
     return J.failed ? -1 : 0;
 }
+
+
+/* ------------------------------------------------------------------------ */
+/* Keep-mask producers.  The radpulse article ("Integrated pack pipeline")   */
+/* notes that the pipeline is independent of the pruning method and names    */
+/* Threshold-l2 among the methods it serves; a score top-k is the other      */
+/* common selector.  The pages give neither rule in detail; the readings are: */
+/*  - Threshold-l2: token j of image b is kept when the Euclidean norm of its */
+/*    feature vector is at least tau;                                        */
+/*  - top-k: image b keeps its CLS token and the k_b - 1 other tokens with   */
+/*    the highest scores, ties going to the lower index and NaN ranking      */
+/*    below every number; k_b is clamped to [1, L_full].                     */
+/* CLS (index 0) is always kept, as everywhere in the pipeline.              */
+/* ------------------------------------------------------------------------ */
+
+/* Does score a (token ia) rank before score b (token ib)? */
+static int ranks_before(float a, int64_t ia, float b, int64_t ib)
+{
+    int na = isnan(a) != 0, nb = isnan(b) != 0;
+    if (na != nb)
+        return nb; /* every number ranks before NaN */
+    if (!na && a != b)
+        return a > b;
+    return ia < ib;
+}
+
+/* keep [B, L_full] <- the top-k selection above; scores is [B, L_full]. */
+void oracle_mask_topk(const float *scores, int64_t B, int64_t L_full, const int32_t *keep_count,
+                      uint8_t *keep)
+{
+    int64_t *order = (int64_t *)malloc(sizeof(int64_t) * (size_t)(L_full > 0 ? L_full : 1));
+    for (int64_t b = 0; b < B; ++b) {
+        const float *s = scores + b * L_full;
+        /* non-CLS tokens in rank order, by insertion */
+        int64_t n = 0;
+        for (int64_t j = 1; j < L_full; ++j) {
+            int64_t pos = n;
+            while (pos > 0 && ranks_before(s[j], j, s[order[pos - 1]], order[pos - 1])) {
+                order[pos] = order[pos - 1];
+                --pos;
+            }
+            order[pos] = j;
+            ++n;
+        }
+        int64_t k = keep_count[b];
+        if (k < 1)
+            k = 1;
+        if (k > L_full)
+            k = L_full;
+        memset(keep + b * L_full, 0, (size_t)L_full);
+        keep[b * L_full] = 1;
+        for (int64_t r = 0; r < k - 1; ++r)
+            keep[b * L_full + order[r]] = 1;
+    }
+    free(order);
+}
+
+/* keep [B, L_full] <- Threshold-l2 of the tokens of x: token (b, j) is the C
+ * elements starting at element (b * L_full + j) * tok_stride.  The sum of
+ * squares is exact up to fp64 rounding (every square of an f16, bf16 or f32
+ * element is exact in fp64).  Where it decides a keep bit, both sides must
+ * round the same additions, so the sum is formed in the order the GPU kernel
+ * uses: 32 partial sums over the elements c = l, l + 32, l + 64, ... in turn
+ * (l = 0..31), then combined pairwise, partial l with partial l + 16, then
+ * l + 8, l + 4, l + 2, l + 1.  The norm is the correctly rounded square root. */
+void oracle_mask_l2(const void *x, int dtype, int64_t B, int64_t L_full, int64_t C, int64_t tok_stride,
+                    double tau, uint8_t *keep)
+{
+    for (int64_t t = 0; t < B * L_full; ++t) {
+        double part[32];
+        for (int l = 0; l < 32; ++l) {
+            part[l] = 0.0;
+            for (int64_t c = l; c < C; c += 32) {
+                const double v = load_elem(x, dtype, t * tok_stride + c);
+                part[l] = part[l] + v * v;
+            }
+        }
+        for (int off = 16; off >= 1; off >>= 1)
+            for (int l = 0; l < off; ++l)
+                part[l] = part[l] + part[l + off];
+        const int64_t j = t % L_full;
+        keep[t] = (j == 0 || sqrt(part[0]) >= tau) ? 1 : 0;
+    }
+}

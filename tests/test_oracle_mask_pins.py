@@ -1,0 +1,111 @@
+"""Pins for the CPU oracle's keep-mask producers (CPU only).
+
+Readings (the pages name Threshold-l2 among the pruning methods the pipeline
+serves, radpulse "Integrated pack pipeline", without spelling out a rule):
+  top-k      image b keeps CLS and the k_b - 1 other tokens with the highest
+             scores; ties go to the lower index, NaN ranks below every
+             number; k_b is clamped to [1, L_full];
+  l2         token kept when the Euclidean norm of its features is >= tau;
+             CLS is always kept.
+Each pin ties the oracle to something other than itself: a sort by numpy's
+lexsort, exact rational arithmetic, closed cases and invariants.
+"""
+from fractions import Fraction
+
+import numpy as np
+import pytest
+
+import oracle
+import synthetic
+
+
+def _topk_by_lexsort(scores, k):
+    B, L = scores.shape
+    keep = np.zeros((B, L), dtype=np.uint8)
+    for b in range(B):
+        s = scores[b, 1:].astype(np.float64)
+        nan = np.isnan(s)
+        key_score = np.where(nan, 0.0, -s)                 # descending score
+        order = np.lexsort((np.arange(1, L), key_score, nan))  # numbers first, then score, then index
+        kk = int(min(max(k[b], 1), L))
+        keep[b, 0] = 1
+        keep[b, 1 + order[:kk - 1]] = 1
+    return keep
+
+
+def _random_scores(rng, B, L, ties=False, nans=False):
+    s = rng.standard_normal((B, L)).astype(np.float32)
+    if ties:
+        s = np.round(s * 2) / 2                            # many exact ties
+    if nans:
+        s[rng.random((B, L)) < 0.1] = np.nan
+    return s
+
+
+@pytest.mark.parametrize("ties,nans", [(False, False), (True, False), (False, True), (True, True)])
+def test_topk_matches_lexsort(ties, nans):
+    rng = synthetic.rng_for(2001, int(ties) * 2 + int(nans))
+    B, L = 7, 97
+    s = _random_scores(rng, B, L, ties, nans)
+    k = rng.integers(-2, L + 5, size=B).astype(np.int32)   # includes out-of-range counts
+    assert np.array_equal(oracle.mask_topk(s, k), _topk_by_lexsort(s, k))
+
+
+def test_topk_closed_cases():
+    s = np.array([[0.0, 3.0, 1.0, 2.0, 3.0, np.nan]], dtype=np.float32)
+    # top-2 of indices 1..5: the two 3.0s (tie: lower index first is irrelevant, both kept)
+    assert oracle.mask_topk(s, np.array([3])).tolist() == [[1, 1, 0, 0, 1, 0]]
+    # top-1: the lower-index 3.0
+    assert oracle.mask_topk(s, np.array([2])).tolist() == [[1, 1, 0, 0, 0, 0]]
+    # k = 1: CLS only; k >= L: everything, NaN included
+    assert oracle.mask_topk(s, np.array([1])).tolist() == [[1, 0, 0, 0, 0, 0]]
+    assert oracle.mask_topk(s, np.array([99])).tolist() == [[1, 1, 1, 1, 1, 1]]
+    # the NaN token is the last one chosen
+    assert oracle.mask_topk(s, np.array([5])).tolist() == [[1, 1, 1, 1, 1, 0]]
+    # CLS's own score never matters
+    s2 = s.copy()
+    s2[0, 0] = -np.inf
+    assert np.array_equal(oracle.mask_topk(s2, np.array([3])), oracle.mask_topk(s, np.array([3])))
+
+
+def test_topk_counts_and_cls():
+    rng = synthetic.rng_for(2002)
+    s = _random_scores(rng, 16, 197, nans=True)
+    k = rng.integers(1, 197, size=16).astype(np.int32)
+    keep = oracle.mask_topk(s, k)
+    assert np.all(keep[:, 0] == 1)
+    assert np.array_equal(keep.sum(1), k)
+
+
+def _exact_norm_sq(row_values):
+    return sum(Fraction(float(v)) ** 2 for v in row_values)
+
+
+@pytest.mark.parametrize("dtype", ["f16", "bf16", "f32"])
+def test_l2_matches_exact_arithmetic(dtype):
+    rng = synthetic.rng_for(2003, ["f16", "bf16", "f32"].index(dtype))
+    B, L, C = 3, 41, 70
+    x = synthetic.store(rng.standard_normal((B, L, C)).astype(np.float32), dtype)
+    xf = oracle.decode(x, dtype).reshape(B, L, C)
+    norms = np.sqrt(np.sum(xf * xf, axis=2))
+    tau = float(np.median(norms))
+    keep = oracle.mask_l2(x, dtype, tau)
+    tau_sq = Fraction(tau) ** 2
+    for b in range(B):
+        for j in range(L):
+            want = 1 if j == 0 or _exact_norm_sq(xf[b, j]) >= tau_sq else 0
+            assert keep[b, j] == want, (b, j)
+
+
+def test_l2_boundary_and_closed_cases():
+    # norm exactly tau (3-4-5 and 5-12-13) is kept; a hair below is not
+    x = np.zeros((1, 5, 64), dtype=np.float32)
+    x[0, 1, 0], x[0, 1, 40] = 3.0, 4.0            # norm 5, elements in different partial sums
+    x[0, 2, 7], x[0, 2, 39] = 5.0, 12.0           # norm 13
+    x[0, 3, 0] = np.nextafter(np.float32(5.0), np.float32(0.0))
+    x[0, 4, :] = 0.625                            # norm 0.625 * 8 = 5
+    assert oracle.mask_l2(x, "f32", 5.0).tolist() == [[1, 1, 1, 0, 1]]
+    assert oracle.mask_l2(x, "f32", 13.0).tolist() == [[1, 0, 1, 0, 0]]
+    # CLS is kept even with zero features; tau <= 0 keeps everything
+    assert oracle.mask_l2(np.zeros((2, 3, 8), np.float32), "f32", 1.0).tolist() == [[1, 0, 0], [1, 0, 0]]
+    assert oracle.mask_l2(np.zeros((2, 3, 8), np.float32), "f32", 0.0).tolist() == [[1, 1, 1], [1, 1, 1]]

@@ -13,6 +13,7 @@ import numpy as np
 import pytest
 
 import oracle
+import test_oracle_mask_pins as mpins
 import test_oracle_pins as pins
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "ragged_oracle.c")
@@ -32,6 +33,13 @@ MUTANTS = {
                       "        cu[b + 1] = (int32_t)t + 1;\n    }\n    return t;\n}\n\n/* Pack"),
     "pack_reads_wrong_row": ("dense + (b * L_full + j) * row_bytes,\n                       (size_t)row_bytes);\n                ++t;\n            }\n        }\n        cu[b + 1]",
                              "dense + (b * L_full + (L_full - 1 - j)) * row_bytes,\n                       (size_t)row_bytes);\n                ++t;\n            }\n        }\n        cu[b + 1]"),
+    "topk_tie_to_higher_index": ("    return ia < ib;", "    return ia > ib;"),
+    "topk_nan_ranks_first": ("return nb; /* every number ranks before NaN */", "return na; /* every number ranks before NaN */"),
+    "topk_ascending": ("        return a > b;", "        return a < b;"),
+    "topk_one_too_many": ("for (int64_t r = 0; r < k - 1; ++r)", "for (int64_t r = 0; r < k; ++r)"),
+    "l2_strict_threshold": ("sqrt(part[0]) >= tau", "sqrt(part[0]) > tau"),
+    "l2_last_element_dropped": ("for (int64_t c = l; c < C; c += 32)", "for (int64_t c = l; c < C - 1; c += 32)"),
+    "l2_cls_not_forced": ("keep[t] = (j == 0 || sqrt(part[0]) >= tau) ? 1 : 0;", "keep[t] = (sqrt(part[0]) >= tau) ? 1 : 0;"),
 }
 
 
@@ -46,6 +54,12 @@ def _pin_calls():
     for keep in pins._random_masks():
         calls.append(lambda keep=keep: pins.test_seqlens_matches_flatnonzero(keep))
         calls.append(lambda keep=keep: pins.test_pack_unpack_roundtrip(keep))
+    calls += [mpins.test_topk_closed_cases, mpins.test_topk_counts_and_cls, mpins.test_l2_boundary_and_closed_cases]
+    for ties in (False, True):
+        for nans in (False, True):
+            calls.append(lambda ties=ties, nans=nans: mpins.test_topk_matches_lexsort(ties, nans))
+    for dt in ("f16", "bf16", "f32"):
+        calls.append(lambda dt=dt: mpins.test_l2_matches_exact_arithmetic(dt))
     return calls
 
 
