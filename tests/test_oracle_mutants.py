@@ -36,7 +36,7 @@ MUTANTS = {
     "topk_tie_to_higher_index": ("    return ia < ib;", "    return ia > ib;"),
     "topk_nan_ranks_first": ("return nb; /* every number ranks before NaN */", "return na; /* every number ranks before NaN */"),
     "topk_ascending": ("        return a > b;", "        return a < b;"),
-    "topk_one_too_many": ("for (int64_t r = 0; r < k - 1; ++r)", "for (int64_t r = 0; r < k; ++r)"),
+    "topk_one_too_few": ("for (int64_t r = 0; r < k - 1; ++r)", "for (int64_t r = 0; r < k - 2; ++r)"),
     "l2_strict_threshold": ("sqrt(part[0]) >= tau", "sqrt(part[0]) > tau"),
     "l2_last_element_dropped": ("for (int64_t c = l; c < C; c += 32)", "for (int64_t c = l; c < C - 1; c += 32)"),
     "l2_cls_not_forced": ("keep[t] = (j == 0 || sqrt(part[0]) >= tau) ? 1 : 0;", "keep[t] = (sqrt(part[0]) >= tau) ? 1 : 0;"),
