@@ -452,6 +452,10 @@ def run_ours(args, rank, world, dist):
     # ---- padded PyTorch SDPA baseline, same calls, same synchronisation ----
     padded = padded_baseline(args, pipes, workloads, ncopies, stream)
 
+    # ---- other attention paths on the same calls, and the mask producers ----
+    comps = comparators(args, pipes, workloads, stream) if world == 1 and not args.quick else None
+    masks = mask_producers() if world == 1 and not args.quick else None
+
     # ---- CPU oracle on a bounded sample (rank 0, one GPU only) ----
     cpu = None
     if rank == 0 and world == 1 and not args.quick:
@@ -477,6 +481,8 @@ def run_ours(args, rank, world, dist):
           "direct_call_us_per_call": round(direct_us, 3),
           "per_case": detail,
           "padded_sdpa": padded,
+          "comparators": comps,
+          "mask_producers": masks,
           "larger_workloads_attention": larger,
           "clocks": clocks,
           "cpu_baseline": cpu}
@@ -518,6 +524,125 @@ def padded_baseline(args, pipes, workloads, ncopies, stream):
         ref = pipes[0][i].cls_out.float()
         err = float((call(pipes[0][i], int(workloads[0][i].Lmax)).float() - ref).abs().max())
         res[f"b{B}_p{int(p * 100)}"] = {"total_us": round(statistics.median(tot), 2), "max_abs_vs_ragged": err}
+    return res
+
+
+def comparators(args, pipes, workloads, stream):
+    """Other ways to run the same per-sequence attention on the serving calls,
+    each call synchronised like ours (median µs):
+      varlen_attn         torch.nn.attention.varlen.varlen_attn (FlashAttention
+                          varlen, the pages' FA2 comparator) on the packed q/k/v
+                          of the same call, plus the CLS gather;
+      nested_sdpa         scaled_dot_product_attention on jagged NestedTensors
+                          built from the same packed q/k/v and cu_seqlens;
+      torch_varlen_path   the whole call in PyTorch: keep mask -> nonzero (a
+                          host sync) -> row gather -> cumsum cu_seqlens ->
+                          varlen_attn -> CLS.
+    max_abs_vs_ragged compares each CLS result with ours."""
+    import torch
+    import torch.nn.functional as F
+    import ragged_variable_length_b200 as rv
+    try:
+        from torch.nn.attention.varlen import varlen_attn
+    except ImportError:
+        varlen_attn = None
+    reps = max(20, min(200, args.steps))
+
+    def timed(fn):
+        tot = []
+        for r in range(reps + 3):
+            torch.cuda.synchronize()
+            t0 = time.perf_counter()
+            fn()
+            stream.synchronize()
+            if r >= 3:
+                tot.append((time.perf_counter() - t0) * 1e6)
+        return round(statistics.median(tot), 2)
+
+    res = {}
+    for i, (B, p) in enumerate(CASES):
+        w, pl = workloads[0][i], pipes[0][i]
+        H, d = w.H, w.d
+        packed, cu = rv.ragged_pack(pl.dense_qkv, pl.keep)
+        T, Lmax = int(w.lengths.sum()), int(w.Lmax)
+        q, k, v = (packed[:T, j].contiguous() for j in range(3))
+        first = cu[:-1].long()
+        ref = pl.cls_out.float()
+        entry = {}
+        cases = {}
+        if varlen_attn is not None:
+            cases["varlen_attn"] = lambda: varlen_attn(q, k, v, cu, cu, Lmax, Lmax, scale=0.125)[first]
+
+            def native():
+                keep = pl.keep.bool()
+                keep[:, 0] = True
+                idx = keep.flatten().nonzero().squeeze(1)
+                rows = pl.dense_qkv.view(-1, 3, H, d).index_select(0, idx)
+                cuv = torch.zeros(B + 1, dtype=torch.int32, device=rows.device)
+                cuv[1:] = torch.cumsum(keep.sum(1, dtype=torch.int32), 0)
+                o = varlen_attn(rows[:, 0].contiguous(), rows[:, 1].contiguous(), rows[:, 2].contiguous(), cuv, cuv,
+                                Lmax, Lmax, scale=0.125)
+                return o[cuv[:-1].long()]
+            cases["torch_varlen_path"] = native
+
+        def nested():
+            offs = cu.long()
+            qn, kn, vn = (torch.nested.nested_tensor_from_jagged(x, offs).transpose(1, 2) for x in (q, k, v))
+            o = F.scaled_dot_product_attention(qn, kn, vn, scale=0.125)
+            return o.transpose(1, 2).values()[first]
+        cases["nested_sdpa"] = nested
+        for name, fn in cases.items():
+            try:
+                err = float((fn().float() - ref).abs().max())
+                entry[name] = {"total_us": timed(fn), "max_abs_vs_ragged": err}
+            except Exception as e:   # an unsupported path on this torch build is reported, not fatal
+                entry[name] = {"unavailable": f"{type(e).__name__}: {str(e)[:120]}"}
+        res[f"b{B}_p{int(p * 100)}"] = entry
+        del packed, q, k, v
+    return res
+
+
+def mask_producers():
+    """Device time per launch of the keep-mask producers, from a CUDA graph of
+    50 back-to-back launches between two events: ragged_pack_topk (top-k
+    selection fused into pack), ragged_mask_l2 (Threshold-l2 over the q
+    features of each token) and, for reference, ragged_pack with a given
+    mask, on a serving batch and on the B=512 sweep shape."""
+    import torch
+    import ragged_variable_length_b200 as rv
+    res = {}
+    for name, w in (("serving_b4", synthetic.serving(4, 0.5)), ("sweep_b512", synthetic.sweep(0.5))):
+        rng = synthetic.rng_for(4001)
+        dense = torch.from_numpy(w.qkv.view(np.int16)).cuda().view(torch.float16)
+        scores = torch.from_numpy(rng.standard_normal((w.B, w.L_full)).astype(np.float32)).cuda()
+        kc = torch.from_numpy(w.lengths.astype(np.int32)).cuda()
+        packed = torch.empty((w.B * w.L_full, 3, w.H, 64), dtype=torch.float16, device="cuda")
+        cu = torch.empty(w.B + 1, dtype=torch.int32, device="cuda")
+        keep = torch.empty((w.B, w.L_full), dtype=torch.uint8, device="cuda")
+        qfeat = dense.view(w.B, w.L_full, 3 * w.H * 64)[:, :, :w.H * 64]
+        keep_given = torch.from_numpy(w.keep).cuda()
+        out = {}
+        for kname, fn in (("pack_topk", lambda: rv.ragged_pack_topk(dense, scores, kc, packed=packed, cu_seqlens=cu)),
+                          ("mask_l2", lambda: rv.ragged_mask_l2(qfeat, 8.0, keep=keep)),
+                          ("pack_given_mask", lambda: rv.ragged_pack(dense, keep_given, packed=packed,
+                                                                     cu_seqlens=cu))):
+            for _ in range(3):
+                fn()
+            torch.cuda.synchronize()
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                for _ in range(50):
+                    fn()
+            graph.replay()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            graph.replay()
+            e1.record()
+            torch.cuda.synchronize()
+            out[kname] = round(e0.elapsed_time(e1) * 1000 / 50, 2)
+            del graph
+        res[name] = {"us_per_launch": out, "B": w.B, "L_full": w.L_full, "row_bytes": w.row_bytes}
     return res
 
 

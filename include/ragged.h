@@ -168,6 +168,50 @@ RAGGED_API ragged_status ragged_attn_fwd(const void *q, const void *k, const voi
 RAGGED_API int32_t ragged_set_attn_kernel(int32_t kernel);
 
 /*
+ * ragged_mask_l2 - Threshold-l2 keep mask (a device-side mask producer).
+ * Paper: radpulse section "Integrated pack pipeline" (the pipeline is
+ * independent of the pruning method; Threshold-l2 is among those named).  The
+ * pages give no rule; the reading: token j of image b is kept when the
+ * Euclidean norm of its feature vector is at least tau, and CLS always.
+ *
+ *   x           device, token (b, j) is the C elements starting at element
+ *               (b * L_full + j) * tok_stride; f16, bf16 or f32 (dtype),
+ *               aligned to its element size.  Read only.
+ *   B, L_full   as for ragged_pack (B * L_full < 2^31).
+ *   C           elements per token, 1 <= C <= 2^24; tok_stride >= C.
+ *   tau         threshold, not NaN; tau <= 0 keeps every token.
+ *   keep        device uint8 [B, L_full]: 1 kept, 0 dropped (an input for
+ *               ragged_pack / ragged_pipeline).
+ * The sum of squares is formed in fp64 in a fixed order (lane l of a warp sums
+ * the squares of elements l, l + 32, ..., then the 32 partials are combined
+ * pairwise: 16, 8, 4, 2, 1) and compared as a correctly rounded square root,
+ * so the decision is reproducible bit for bit.
+ */
+RAGGED_API ragged_status ragged_mask_l2(const void *x, int64_t B, int64_t L_full, int64_t C, int64_t tok_stride,
+                                        ragged_dtype dtype, double tau, uint8_t *keep, void *stream);
+
+/*
+ * ragged_pack_topk - score top-k selection fused into pack: one launch
+ * produces the keep decision, cu_seqlens and the packed rows.
+ * Paper: as ragged_pack, and the mask-producer reading above: image b keeps
+ * CLS and the k_b - 1 other tokens with the highest scores (ties: the lower
+ * index; NaN ranks below every number); k_b = keep_count[b] clamped to
+ * [1, L_full], so cu[b + 1] = cu[b] + k_b.
+ *
+ *   dense, B, L_full, row_bytes, packed, cu_seqlens, src_idx: as ragged_pack.
+ *   scores      device float32 [B, L_full], 4-byte aligned; scores[b, 0]
+ *               (CLS) is not used.
+ *   keep_count  device int32 [B]: survivors per image, CLS included.
+ *   keep_out    device uint8 [B, L_full] or NULL: receives the selection
+ *               (for ragged_unpack).
+ * Selection costs O(L_full^2) comparisons per image (meant for ViT token
+ * counts); L_full is limited to 8192 here.
+ */
+RAGGED_API ragged_status ragged_pack_topk(const void *dense, int64_t B, int64_t L_full, int64_t row_bytes,
+                                          const float *scores, const int32_t *keep_count, void *packed,
+                                          int32_t *cu_seqlens, int32_t *src_idx, uint8_t *keep_out, void *stream);
+
+/*
  * ragged_unpack_cls - CLS extraction (step 3).
  * Paper: radpulse section "Integrated pack pipeline" (after attention and the
  * MLP run on the packed tokens, the CLS token is extracted).

@@ -43,13 +43,15 @@ RAGGED_ATTN_STREAMING = 1
 RAGGED_ATTN_RESIDENT = 2
 RAGGED_ATTN_TCGEN05 = 3
 RAGGED_ATTN_PERSISTENT = 4
+RAGGED_F16, RAGGED_BF16, RAGGED_F32 = 0, 1, 2
 
 DTYPE_CODES = {torch.float16: 0, torch.bfloat16: 1, torch.float32: 2}
 DTYPE_NAMES = {"f16": torch.float16, "bf16": torch.bfloat16, "f32": torch.float32}
 
 EXPORTS = ("ragged_pack", "ragged_attn_fwd", "ragged_unpack_cls", "ragged_unpack",
            "ragged_pipeline", "ragged_get_device_status", "ragged_status_string",
-           "ragged_last_error", "ragged_abi_version", "ragged_set_attn_kernel")
+           "ragged_last_error", "ragged_abi_version", "ragged_set_attn_kernel",
+           "ragged_mask_l2", "ragged_pack_topk")
 
 
 class RaggedError(RuntimeError):
@@ -74,6 +76,8 @@ def load(path: Optional[str] = None):
     lib.ragged_pack.argtypes = [vp, i64, i64, i64, vp, vp, vp, vp, vp]
     lib.ragged_attn_fwd.argtypes = [vp, vp, vp, i64, i64, vp, i64, i64, i64, i64, f32, i32, vp, i64, vp, vp]
     lib.ragged_unpack_cls.argtypes = [vp, vp, i64, i64, vp, vp]
+    lib.ragged_mask_l2.argtypes = [vp, i64, i64, i64, i64, i32, ctypes.c_double, vp, vp]
+    lib.ragged_pack_topk.argtypes = [vp, i64, i64, i64, vp, vp, vp, vp, vp, vp, vp]
     lib.ragged_unpack.argtypes = [vp, vp, vp, i64, i64, i64, vp, vp]
     lib.ragged_pipeline.argtypes = [vp, vp, i64, i64, i64, i64, f32, i32, vp, vp, vp, vp, ctypes.c_uint32, vp]
     lib.ragged_get_device_status.argtypes = [ctypes.POINTER(ctypes.c_uint32), vp]
@@ -156,6 +160,42 @@ def ragged_pack(dense: torch.Tensor, keep: torch.Tensor, packed: Optional[torch.
         cu_seqlens = torch.empty(B + 1, dtype=torch.int32, device=dense.device)
     _check(load().ragged_pack(_ptr(dense), B, L_full, row_bytes, _ptr(keep), _ptr(packed),
                               _ptr(cu_seqlens), _ptr(src_idx), _stream(stream)))
+    return packed, cu_seqlens
+
+
+def ragged_mask_l2(x: torch.Tensor, tau: float, keep: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Threshold-l2 keep mask of x [B, L_full, C] (f16 / bf16 / f32, unit stride
+    along C): keep[b, j] = 1 when ||x[b, j]||_2 >= tau, and always for j = 0."""
+    B, L_full, C = x.shape
+    if x.stride(2) != 1 or x.stride(0) != L_full * x.stride(1):
+        raise ValueError("x must be [B, L_full, C] with unit stride along C and tokens evenly spaced")
+    if keep is None:
+        keep = torch.empty((B, L_full), dtype=torch.uint8, device=x.device)
+    _check(load().ragged_mask_l2(_ptr(x), B, L_full, C, x.stride(1), _dtype_code(x), float(tau), _ptr(keep),
+                                 _stream(stream)))
+    return keep
+
+
+def ragged_pack_topk(dense: torch.Tensor, scores: torch.Tensor, keep_count: torch.Tensor,
+                     packed: Optional[torch.Tensor] = None, cu_seqlens: Optional[torch.Tensor] = None,
+                     src_idx: Optional[torch.Tensor] = None, keep_out: Optional[torch.Tensor] = None, stream=None):
+    """Top-k selection fused into pack.  dense [B, L_full, ...] contiguous, scores
+    float32 [B, L_full], keep_count int32 [B] (survivors per image, CLS included)
+    -> (packed, cu_seqlens); keep_out (uint8 [B, L_full]) receives the selection."""
+    B, L_full = int(scores.shape[0]), int(scores.shape[1])
+    if not dense.is_contiguous() or tuple(dense.shape[:2]) != (B, L_full):
+        raise ValueError("dense must be contiguous [B, L_full, ...]")
+    if scores.dtype != torch.float32 or not scores.is_contiguous():
+        raise ValueError("scores must be contiguous float32 [B, L_full]")
+    if keep_count.dtype != torch.int32 or keep_count.numel() != B:
+        raise ValueError("keep_count must be int32 [B]")
+    row_bytes = dense.element_size() * (dense[0, 0].numel() if B else int(torch.tensor(dense.shape[2:]).prod()))
+    if packed is None:
+        packed = torch.empty((B * L_full,) + tuple(dense.shape[2:]), dtype=dense.dtype, device=dense.device)
+    if cu_seqlens is None:
+        cu_seqlens = torch.empty(B + 1, dtype=torch.int32, device=dense.device)
+    _check(load().ragged_pack_topk(_ptr(dense), B, L_full, row_bytes, _ptr(scores), _ptr(keep_count), _ptr(packed),
+                                   _ptr(cu_seqlens), _ptr(src_idx), _ptr(keep_out), _stream(stream)))
     return packed, cu_seqlens
 
 

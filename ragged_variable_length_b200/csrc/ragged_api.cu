@@ -19,6 +19,7 @@
 #include <cudaTypedefs.h>
 #include <mutex>
 #include "common.cuh"
+#include "mask.cuh"
 #include "pack.cuh"
 
 namespace {
@@ -103,7 +104,9 @@ int pack_splits(int64_t B, int64_t L_full) {
     return static_cast<int>(s);
 }
 
-bool g_pack_smem[kMaxDevices], g_unpack_smem[kMaxDevices];
+bool g_pack_smem[kMaxDevices], g_unpack_smem[kMaxDevices], g_topk_smem[kMaxDevices];
+// Largest L_full of the fused top-k pack: scores and survivor list in shared memory.
+constexpr int kTopkMaxTokens = 8192;
 bool g_mma_f16_smem[kMaxDevices], g_mma_bf16_smem[kMaxDevices], g_f32_smem[kMaxDevices];
 
 // Largest dynamic shared memory of the resident kernels: 640 keys and a
@@ -326,6 +329,66 @@ ragged_status ragged_pack(const void* dense, int64_t B, int64_t L_full, int64_t 
         static_cast<const uint4*>(dense), static_cast<int>(L_full),
         static_cast<uint32_t>(row_bytes / 16), keep, static_cast<uint4*>(packed), cu_seqlens, src_idx);
     return cuda_check(cudaGetLastError(), "pack launch");
+}
+
+ragged_status ragged_mask_l2(const void* x, int64_t B, int64_t L_full, int64_t C, int64_t tok_stride,
+                             ragged_dtype dtype, double tau, uint8_t* keep, void* stream) {
+    if (B < 0) return fail(RAGGED_ERR_INVALID_ARG, "B = %lld is negative", (long long)B);
+    if (L_full < 1 || L_full > RAGGED_MAX_TOKENS)
+        return fail(RAGGED_ERR_INVALID_ARG, "L_full = %lld outside [1, %d]", (long long)L_full, RAGGED_MAX_TOKENS);
+    if (B * L_full >= (int64_t(1) << 31))
+        return fail(RAGGED_ERR_UNSUPPORTED, "B * L_full = %lld does not fit int32 offsets", (long long)(B * L_full));
+    if (C < 1 || C > (int64_t(1) << 24))
+        return fail(RAGGED_ERR_INVALID_ARG, "C = %lld outside [1, 2^24]", (long long)C);
+    if (tok_stride < C) return fail(RAGGED_ERR_INVALID_ARG, "tok_stride must be >= C");
+    if (dtype != RAGGED_F16 && dtype != RAGGED_BF16 && dtype != RAGGED_F32)
+        return fail(RAGGED_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
+    if (tau != tau) return fail(RAGGED_ERR_INVALID_ARG, "tau is NaN");
+    if (B == 0) return RAGGED_OK;
+    if (x == nullptr || keep == nullptr) return fail(RAGGED_ERR_INVALID_ARG, "x and keep must not be NULL");
+    const int64_t esz = dtype == RAGGED_F32 ? 4 : 2;
+    if (reinterpret_cast<uintptr_t>(x) % esz) return fail(RAGGED_ERR_INVALID_ARG, "x is not element-aligned");
+    const int64_t tokens = B * L_full;
+    const unsigned blocks = static_cast<unsigned>((tokens + ragged::kMaskThreads / 32 - 1) / (ragged::kMaskThreads / 32));
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int L = static_cast<int>(L_full), Ci = static_cast<int>(C);
+    if (dtype == RAGGED_F16)
+        ragged::mask_l2_kernel<__half><<<blocks, ragged::kMaskThreads, 0, s>>>(x, tokens, L, Ci, tok_stride, tau, keep);
+    else if (dtype == RAGGED_BF16)
+        ragged::mask_l2_kernel<__nv_bfloat16><<<blocks, ragged::kMaskThreads, 0, s>>>(x, tokens, L, Ci, tok_stride, tau,
+                                                                                      keep);
+    else
+        ragged::mask_l2_kernel<float><<<blocks, ragged::kMaskThreads, 0, s>>>(x, tokens, L, Ci, tok_stride, tau, keep);
+    return cuda_check(cudaGetLastError(), "mask_l2 launch");
+}
+
+ragged_status ragged_pack_topk(const void* dense, int64_t B, int64_t L_full, int64_t row_bytes, const float* scores,
+                               const int32_t* keep_count, void* packed, int32_t* cu_seqlens, int32_t* src_idx,
+                               uint8_t* keep_out, void* stream) {
+    ragged_status st = check_rows(B, L_full, row_bytes);
+    if (st != RAGGED_OK) return st;
+    if (L_full > kTopkMaxTokens)
+        return fail(RAGGED_ERR_UNSUPPORTED, "L_full = %lld exceeds %d for the top-k selection", (long long)L_full,
+                    kTopkMaxTokens);
+    if (cu_seqlens == nullptr) return fail(RAGGED_ERR_INVALID_ARG, "cu_seqlens is NULL");
+    if ((reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) || (reinterpret_cast<uintptr_t>(src_idx) & 3u))
+        return fail(RAGGED_ERR_INVALID_ARG, "cu_seqlens / src_idx must be 4-byte aligned");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (B == 0) return cuda_check(cudaMemsetAsync(cu_seqlens, 0, sizeof(int32_t), s), "cudaMemsetAsync");
+    if (dense == nullptr || scores == nullptr || keep_count == nullptr || packed == nullptr)
+        return fail(RAGGED_ERR_INVALID_ARG, "dense, scores, keep_count and packed must not be NULL");
+    if (!aligned16(dense) || !aligned16(packed))
+        return fail(RAGGED_ERR_INVALID_ARG, "dense and packed must be 16-byte aligned");
+    if ((reinterpret_cast<uintptr_t>(scores) & 3u) || (reinterpret_cast<uintptr_t>(keep_count) & 3u))
+        return fail(RAGGED_ERR_INVALID_ARG, "scores / keep_count must be 4-byte aligned");
+    st = ensure_smem(ragged::pack_topk_kernel, 2 * kTopkMaxTokens * static_cast<int>(sizeof(int)), g_topk_smem);
+    if (st != RAGGED_OK) return st;
+    const int smem = static_cast<int>(2 * L_full * sizeof(int));
+    const dim3 grid(pack_splits(B, L_full), static_cast<unsigned>(B));
+    ragged::pack_topk_kernel<<<grid, ragged::kPackThreads, smem, s>>>(
+        static_cast<const uint4*>(dense), static_cast<int>(L_full), static_cast<uint32_t>(row_bytes / 16), scores,
+        keep_count, static_cast<uint4*>(packed), cu_seqlens, src_idx, keep_out);
+    return cuda_check(cudaGetLastError(), "pack_topk launch");
 }
 
 ragged_status ragged_unpack(const void* packed, const int32_t* cu_seqlens, const uint8_t* keep,

@@ -119,6 +119,48 @@ def test_empty_batch_attention_is_a_noop(lib):
     assert _attn(lib, B=0, q=None, k=None, v=None, out=None, cu=None) == rv.RAGGED_OK
 
 
+@pytest.mark.parametrize("kw,status,needle", [
+    (dict(B=-1), rv.RAGGED_ERR_INVALID_ARG, "negative"),
+    (dict(L_full=0), rv.RAGGED_ERR_INVALID_ARG, "L_full"),
+    (dict(C=0), rv.RAGGED_ERR_INVALID_ARG, "C ="),
+    (dict(tok_stride=10), rv.RAGGED_ERR_INVALID_ARG, "tok_stride"),
+    (dict(dtype=7), rv.RAGGED_ERR_INVALID_ARG, "dtype"),
+    (dict(tau=float("nan")), rv.RAGGED_ERR_INVALID_ARG, "NaN"),
+    (dict(x=None), rv.RAGGED_ERR_INVALID_ARG, "NULL"),
+    (dict(keep=None), rv.RAGGED_ERR_INVALID_ARG, "NULL"),
+    (dict(x=A16 + 1), rv.RAGGED_ERR_INVALID_ARG, "aligned"),
+    (dict(B=40000, L_full=60000), rv.RAGGED_ERR_INVALID_ARG, "L_full"),
+])
+def test_mask_l2_rejects(lib, kw, status, needle):
+    a = dict(x=A16, B=2, L_full=197, C=384, tok_stride=384, dtype=rv.RAGGED_F16, tau=1.0, keep=A16)
+    a.update(kw)
+    assert lib.ragged_mask_l2(a["x"], a["B"], a["L_full"], a["C"], a["tok_stride"], a["dtype"], a["tau"],
+                              a["keep"], None) == status
+    assert needle in rv.ragged_last_error()
+
+
+def test_empty_batch_mask_is_a_noop(lib):
+    assert lib.ragged_mask_l2(None, 0, 197, 384, 384, rv.RAGGED_F16, 1.0, None, None) == rv.RAGGED_OK
+
+
+@pytest.mark.parametrize("kw,status,needle", [
+    (dict(B=-1), rv.RAGGED_ERR_INVALID_ARG, "negative"),
+    (dict(L_full=9000), rv.RAGGED_ERR_UNSUPPORTED, "8192"),
+    (dict(row_bytes=24), rv.RAGGED_ERR_INVALID_ARG, "multiple of 16"),
+    (dict(cu=None), rv.RAGGED_ERR_INVALID_ARG, "cu_seqlens"),
+    (dict(scores=None), rv.RAGGED_ERR_INVALID_ARG, "NULL"),
+    (dict(count=None), rv.RAGGED_ERR_INVALID_ARG, "NULL"),
+    (dict(scores=A16 + 2), rv.RAGGED_ERR_INVALID_ARG, "4-byte"),
+    (dict(dense=A8), rv.RAGGED_ERR_INVALID_ARG, "16-byte"),
+])
+def test_pack_topk_rejects(lib, kw, status, needle):
+    a = dict(dense=A16, B=2, L_full=197, row_bytes=768, scores=A16, count=A16, packed=A16, cu=A16)
+    a.update(kw)
+    assert lib.ragged_pack_topk(a["dense"], a["B"], a["L_full"], a["row_bytes"], a["scores"], a["count"],
+                                a["packed"], a["cu"], None, None, None) == status
+    assert needle in rv.ragged_last_error()
+
+
 def test_unpack_rejects(lib):
     assert lib.ragged_unpack(A16, A16, A16, 2, 197, 40, A16, None) == rv.RAGGED_ERR_INVALID_ARG
     assert lib.ragged_unpack(None, A16, A16, 2, 197, 48, A16, None) == rv.RAGGED_ERR_INVALID_ARG

@@ -1,0 +1,108 @@
+"""GPU parity of the device-side keep-mask producers against the CPU oracle.
+
+Readings (the pages name Threshold-l2 among the pruning methods the pipeline
+serves, radpulse "Integrated pack pipeline"; the rules are not spelled out):
+Threshold-l2 keeps a token whose feature norm is >= tau; top-k keeps CLS and
+the k_b - 1 highest-scoring other tokens (ties: lower index, NaN last).  Masks,
+cu_seqlens and packed rows are integer / byte results: bit-exact.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import ragged_variable_length_b200 as rv
+import synthetic
+from helpers import to_device, to_host_bits
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("dtype", ["f16", "bf16", "f32"])
+@pytest.mark.parametrize("B,L,C", [(4, 197, 384), (3, 577, 768), (2, 33, 70)])
+def test_mask_l2_matches_oracle(dtype, B, L, C):
+    rng = synthetic.rng_for(3001, B * 1000 + C)
+    x = synthetic.store(rng.standard_normal((B, L, C)).astype(np.float32), dtype)
+    xf = oracle.decode(x, dtype).reshape(B, L, C)
+    norms = np.sqrt((xf * xf).sum(2))
+    for tau in (float(np.median(norms)), float(norms.min()), float(norms.max()), 0.0):
+        got = rv.ragged_mask_l2(to_device(x, dtype), tau).cpu().numpy()
+        assert np.array_equal(got, oracle.mask_l2(x, dtype, tau)), tau
+
+
+def test_mask_l2_at_the_threshold():
+    x = np.zeros((1, 5, 64), dtype=np.float32)
+    x[0, 1, 0], x[0, 1, 40] = 3.0, 4.0
+    x[0, 2, 7], x[0, 2, 39] = 5.0, 12.0
+    x[0, 3, 0] = np.nextafter(np.float32(5.0), np.float32(0.0))
+    x[0, 4, :] = 0.625
+    for tau in (5.0, 13.0):
+        got = rv.ragged_mask_l2(torch.from_numpy(x).cuda(), tau).cpu().numpy()
+        assert np.array_equal(got, oracle.mask_l2(x, "f32", tau))
+    assert rv.ragged_mask_l2(torch.from_numpy(x).cuda(), 5.0).cpu().tolist() == [[1, 1, 1, 0, 1]]
+
+
+def test_mask_l2_on_a_strided_view():
+    """Norm of the q part of a dense fused [B, L, 3, H, 64] buffer (token stride 3 * H * 64)."""
+    w = synthetic.serving(4, 0.0)
+    dense = to_device(w.qkv, w.dtype)                       # [B, L, 3, H, 64]
+    q = dense.view(w.B, w.L_full, 3 * w.H * 64)[:, :, :w.H * 64]
+    qn = w.qkv[:, :, 0].reshape(w.B, w.L_full, w.H * 64)
+    norms = np.sqrt((oracle.decode(np.ascontiguousarray(qn), w.dtype).reshape(qn.shape) ** 2).sum(2))
+    tau = float(np.median(norms))
+    got = rv.ragged_mask_l2(q, tau).cpu().numpy()
+    assert np.array_equal(got, oracle.mask_l2(np.ascontiguousarray(qn), w.dtype, tau))
+
+
+def _topk_case(rng, B, L, ties, nans):
+    s = rng.standard_normal((B, L)).astype(np.float32)
+    if ties:
+        s = np.round(s * 2) / 2
+    if nans:
+        s[rng.random((B, L)) < 0.1] = np.nan
+    k = rng.integers(-3, L + 4, size=B).astype(np.int32)
+    k[:2] = [1, L]
+    return s, k
+
+
+@pytest.mark.parametrize("B,L,H,dtype", [(4, 197, 6, "f16"), (32, 197, 12, "bf16"), (64, 577, 12, "bf16"),
+                                         (3, 40, 2, "f16")])
+@pytest.mark.parametrize("ties,nans", [(False, False), (True, True)])
+def test_pack_topk_matches_oracle(B, L, H, dtype, ties, nans):
+    rng = synthetic.rng_for(3002, B * 100 + int(ties) * 2 + int(nans))
+    s, k = _topk_case(rng, B, L, ties, nans)
+    qkv = synthetic.store(rng.standard_normal((B, L, 3, H, 64)).astype(np.float32), dtype)
+    dense = to_device(qkv, dtype)
+    keep_out = torch.full((B, L), 7, dtype=torch.uint8, device="cuda")
+    src_idx = torch.full((B * L,), -1, dtype=torch.int32, device="cuda")
+    packed, cu = rv.ragged_pack_topk(dense, torch.from_numpy(s).cuda(), torch.from_numpy(k).cuda(),
+                                     src_idx=src_idx, keep_out=keep_out)
+    torch.cuda.synchronize()
+    keep_ref = oracle.mask_topk(s, k)
+    assert np.array_equal(keep_out.cpu().numpy(), keep_ref)
+    packed_ref, cu_ref = oracle.pack(qkv, keep_ref)
+    cu_h = cu.cpu().numpy()
+    assert np.array_equal(cu_h, cu_ref)
+    T = int(cu_h[-1])
+    assert np.array_equal(to_host_bits(packed[:T], dtype), packed_ref)
+    src_ref = np.concatenate([b * L + np.flatnonzero(keep_ref[b]) for b in range(B)])
+    assert np.array_equal(src_idx[:T].cpu().numpy(), src_ref)
+
+
+def test_pack_topk_then_attention():
+    """Selection, pack and attention chain: the attention of the top-k packed
+    rows equals the oracle's attention of the oracle's selection."""
+    rng = synthetic.rng_for(3003)
+    B, L, H = 8, 197, 6
+    s, _ = _topk_case(rng, B, L, False, False)
+    k = rng.integers(20, 120, size=B).astype(np.int32)
+    w = synthetic.make_workload("topk_chain", B, L, H, k, "f16", 3004)
+    packed, cu = rv.ragged_pack_topk(to_device(w.qkv, "f16"), torch.from_numpy(s).cuda(), torch.from_numpy(k).cuda())
+    out = rv.ragged_attn_fwd(packed[:, 0], packed[:, 1], packed[:, 2], cu, L, 0.125)
+    torch.cuda.synchronize()
+    keep_ref = oracle.mask_topk(s, k)
+    packed_ref, cu_ref = oracle.pack(w.qkv, keep_ref)
+    ref = oracle.attention(packed_ref[:, 0], packed_ref[:, 1], packed_ref[:, 2], cu_ref, "f16", 0.125)
+    T = int(cu_ref[-1])
+    got = out[:T].double().cpu().numpy()
+    assert np.abs(got - ref).max() <= 4e-3
