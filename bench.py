@@ -455,6 +455,7 @@ def run_ours(args, rank, world, dist):
     # ---- other attention paths on the same calls, and the mask producers ----
     comps = comparators(args, pipes, workloads, stream) if world == 1 and not args.quick else None
     masks = mask_producers() if world == 1 and not args.quick else None
+    block = deit_block() if world == 1 and not args.quick else None
 
     # ---- CPU oracle on a bounded sample (rank 0, one GPU only) ----
     cpu = None
@@ -483,6 +484,7 @@ def run_ours(args, rank, world, dist):
           "padded_sdpa": padded,
           "comparators": comps,
           "mask_producers": masks,
+          "deit_block": block,
           "larger_workloads_attention": larger,
           "clocks": clocks,
           "cpu_baseline": cpu}
@@ -643,6 +645,80 @@ def mask_producers():
             out[kname] = round(e0.elapsed_time(e1) * 1000 / 50, 2)
             del graph
         res[name] = {"us_per_launch": out, "B": w.B, "L_full": w.L_full, "row_bytes": w.row_bytes}
+    return res
+
+
+def deit_block():
+    """One random-weight DeiT-S encoder block (D = 384, 6 heads, MLP 1536, f16)
+    on pruned tokens, two ways, each captured as a CUDA graph and timed by
+    replay between events:
+      packed  ragged_pack of the dense tokens -> LayerNorm -> QKV GEMM on the T
+              survivors -> ragged_attn_fwd -> projection -> residual ->
+              LayerNorm -> MLP (GELU) -> residual -> CLS rows (cu_seqlens);
+      padded  survivors gathered to [B, Lmax] (Lmax from the generator) -> the
+              same layers on B * Lmax rows with SDPA under a key-padding mask
+              -> CLS rows.
+    The GEMMs are cuBLAS (torch); T and Lmax come from the host-side
+    generator, so neither path synchronises.  cls_max_abs compares the two."""
+    import torch
+    import torch.nn.functional as F
+    import ragged_variable_length_b200 as rv
+    D, H, d, M, L_full = 384, 6, 64, 1536, 197
+    g = torch.Generator(device="cuda").manual_seed(5001)
+    wt = lambda *shape: (torch.randn(*shape, device="cuda", generator=g) * 0.02).half()
+    Wqkv, Wo, W1, W2 = wt(3 * D, D), wt(D, D), wt(M, D), wt(D, M)
+    res = {}
+    for B, rate in ((32, 0.5), (64, 0.5), (64, 0.0)):
+        rng = synthetic.rng_for(5002, B * 10 + int(rate * 10))
+        lengths = synthetic.serving_lengths(rng, B, rate)
+        keep_np = synthetic.topk_keep_mask(rng, L_full, lengths)
+        x = torch.from_numpy(rng.standard_normal((B, L_full, D)).astype(np.float16)).cuda()
+        keep = torch.from_numpy(keep_np).cuda()
+        T, Lmax = int(lengths.sum()), int(lengths.max())
+        idx = torch.from_numpy(np.stack([np.concatenate([np.flatnonzero(r), np.zeros(Lmax - r.sum(), np.int64)])
+                                         for r in keep_np])).cuda()
+        valid = torch.arange(Lmax, device="cuda")[None, :] < torch.from_numpy(lengths).cuda()[:, None]
+
+        def packed_block():
+            xp, cu = rv.ragged_pack(x, keep)
+            h = xp[:T]
+            qkv = F.linear(F.layer_norm(h, (D,)), Wqkv).view(T, 3, H, d)
+            a = rv.ragged_attn_fwd(qkv[:, 0], qkv[:, 1], qkv[:, 2], cu, L_full, 0.125).view(T, D)
+            h = h + F.linear(a, Wo)
+            h = h + F.linear(F.gelu(F.linear(F.layer_norm(h, (D,)), W1)), W2)
+            return h[cu[:-1].long()]
+
+        def padded_block():
+            h = torch.gather(x, 1, idx[:, :, None].expand(B, Lmax, D))
+            qkv = F.linear(F.layer_norm(h, (D,)), Wqkv).view(B, Lmax, 3, H, d).permute(2, 0, 3, 1, 4)
+            a = F.scaled_dot_product_attention(qkv[0], qkv[1], qkv[2], attn_mask=valid[:, None, None, :])
+            h = h + F.linear(a.transpose(1, 2).reshape(B, Lmax, D), Wo)
+            h = h + F.linear(F.gelu(F.linear(F.layer_norm(h, (D,)), W1)), W2)
+            return h[:, 0]
+
+        entry = {"B": B, "prune_rate": rate, "T": T, "Lmax": Lmax}
+        outs = {}
+        for name, fn in (("packed_us", packed_block), ("padded_us", padded_block)):
+            for _ in range(3):
+                fn()
+            torch.cuda.synchronize()
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                out = fn()
+            graph.replay()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(20):
+                graph.replay()
+            e1.record()
+            torch.cuda.synchronize()
+            entry[name] = round(e0.elapsed_time(e1) * 1000 / 20, 2)
+            outs[name] = out.float().clone()
+            del graph
+        entry["speedup"] = round(entry["padded_us"] / entry["packed_us"], 3)
+        entry["cls_max_abs"] = float((outs["packed_us"] - outs["padded_us"]).abs().max())
+        res[f"b{B}_p{int(rate * 100)}"] = entry
     return res
 
 
