@@ -204,8 +204,9 @@ RAGGED_API ragged_status ragged_mask_l2(const void *x, int64_t B, int64_t L_full
  *   keep_count  device int32 [B]: survivors per image, CLS included.
  *   keep_out    device uint8 [B, L_full] or NULL: receives the selection
  *               (for ragged_unpack).
- * Selection costs O(L_full^2) comparisons per image (meant for ViT token
- * counts); L_full is limited to 8192 here.
+ * Each CTA sorts its image's scores in shared memory (a bitonic network over
+ * L_full rounded up to a power of two); -0 and +0 tie, NaNs of any payload
+ * tie.  L_full is limited to 8192 here (RAGGED_ERR_UNSUPPORTED above it).
  */
 RAGGED_API ragged_status ragged_pack_topk(const void *dense, int64_t B, int64_t L_full, int64_t row_bytes,
                                           const float *scores, const int32_t *keep_count, void *packed,

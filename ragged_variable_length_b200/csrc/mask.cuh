@@ -11,7 +11,7 @@
 //
 // mask_l2_kernel writes a keep mask for ragged_pack.  pack_topk_kernel is the
 // top-k selection fused into pack: since image b keeps exactly k_b tokens,
-// cu[b] is the sum of the earlier k_b, and each CTA ranks its image's scores
+// cu[b] is the sum of the earlier k_b, and each CTA sorts its image's scores
 // itself, so selection, cu_seqlens and the survivor copy are one launch.
 #pragma once
 
@@ -36,6 +36,8 @@ __device__ __forceinline__ double widen<float>(const void* p, int64_t i) {
 
 constexpr int kMaskThreads = 256;   // 8 tokens per CTA, one warp each
 
+constexpr int kMaskBatch = 16;      // loads in flight per lane before they are summed
+
 // keep[t] for the tokens t = 0 .. tokens - 1 (t = b * L_full + j) of x, token t
 // being the C elements from element t * tok_stride.  The sum of squares is
 // formed in fp64 in a fixed order, so that the keep decision at the threshold
@@ -43,7 +45,9 @@ constexpr int kMaskThreads = 256;   // 8 tokens per CTA, one warp each
 // in turn (every square of an f16, bf16 or f32 element is exact in fp64), then
 // the 32 partial sums are combined pairwise with xor-shuffles 16, 8, 4, 2, 1.
 // Explicit round-to-nearest intrinsics keep the compiler from contracting the
-// multiply-add.
+// multiply-add.  Elements are loaded kMaskBatch at a time before any is
+// added; slots past C load 0, and adding +0 to the (non-negative) sum leaves
+// it unchanged, so the batching does not alter the order's result.
 template <typename T>
 __global__ void __launch_bounds__(kMaskThreads)
     mask_l2_kernel(const void* __restrict__ x, int64_t tokens, int L_full, int C, int64_t tok_stride, double tau,
@@ -53,37 +57,64 @@ __global__ void __launch_bounds__(kMaskThreads)
     if (t >= tokens) return;   // warp-uniform
     const int64_t base = t * tok_stride;
     double ss = 0.0;
-    for (int c = lane; c < C; c += 32) {
-        const double v = widen<T>(x, base + c);
-        ss = __dadd_rn(ss, __dmul_rn(v, v));
+    for (int c0 = 0; c0 < C; c0 += 32 * kMaskBatch) {
+        double v[kMaskBatch];
+#pragma unroll
+        for (int u = 0; u < kMaskBatch; ++u) {
+            const int c = c0 + 32 * u + lane;
+            v[u] = c < C ? widen<T>(x, base + c) : 0.0;
+        }
+#pragma unroll
+        for (int u = 0; u < kMaskBatch; ++u) ss = __dadd_rn(ss, __dmul_rn(v[u], v[u]));
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) ss = __dadd_rn(ss, __shfl_xor_sync(0xffffffffu, ss, off));
     if (lane == 0) keep[t] = (t % L_full == 0 || __dsqrt_rn(ss) >= tau) ? 1 : 0;
 }
 
-// Does score a (token ia) rank before score b (token ib)?
-__device__ __forceinline__ bool ranks_before(float a, int ia, float b, int ib) {
-    const bool na = isnan(a), nb = isnan(b);
-    if (na != nb) return nb;   // every number ranks before NaN
-    if (!na && a != b) return a > b;
-    return ia < ib;
+// The top-k order as one unsigned key per token, larger key = ranks earlier:
+// the high word maps the score's bits so that unsigned order is float order
+// (-0 folded onto +0, so the two zeros tie) and sends NaN, of any payload, to 0
+// below -inf; the low word is ~j, so equal scores go to the lower index.  Keys
+// of distinct tokens differ, and every token j < 2^31 has a key above 0.
+// Integer operations only, so no flush-to-zero setting can merge scores.
+__device__ __forceinline__ uint64_t topk_key(float score, int j) {
+    uint32_t bits = __float_as_uint(score);
+    const uint32_t mag = bits & 0x7fffffffu;
+    uint32_t hi;
+    if (mag > 0x7f800000u) {
+        hi = 0u;                                    // NaN
+    } else {
+        if (mag == 0u) bits = 0u;                   // -0 -> +0
+        hi = (bits & 0x80000000u) ? ~bits : (bits | 0x80000000u);
+    }
+    return (static_cast<uint64_t>(hi) << 32) | static_cast<uint32_t>(~static_cast<uint32_t>(j));
 }
 
 __device__ __forceinline__ int clamp_count(int k, int L_full) { return k < 1 ? 1 : (k > L_full ? L_full : k); }
 
-// grid = (splits, B).  Dynamic shared memory: L_full scores, then L_full ints
-// of survivor list.  Each CTA ranks image b's non-CLS tokens against each other
-// (O(L_full^2 / threads) comparisons; fine for ViT token counts), builds the
-// survivor list in token order with the ballot scan of pack, and copies its
-// slice of rows.  Split 0 also writes cu[b + 1] and, when asked, the keep row.
+__host__ __device__ constexpr int topk_pow2(int n) {
+    int p = 2;
+    while (p < n) p <<= 1;
+    return p;
+}
+
+// grid = (splits, B).  Dynamic shared memory: P = topk_pow2(L_full) 8-byte
+// keys, then L_full ints of survivor list.  Each CTA sorts image b's keys in
+// descending order (bitonic network over P slots; CLS and the padding slots
+// hold key 0, which every other token's key exceeds), so the (k_b - 1)-th
+// largest key is the cut: a non-CLS token is kept when its key is at least
+// that.  The survivor list is then built in token order with the ballot scan
+// of pack, and the CTA copies its slice of rows.  Split 0 also writes
+// cu[b + 1] and, when asked, the keep row.
 __global__ void __launch_bounds__(kPackThreads)
     pack_topk_kernel(const uint4* __restrict__ dense, int L_full, uint32_t nvec, const float* __restrict__ scores,
                      const int32_t* __restrict__ keep_count, uint4* __restrict__ packed, int32_t* __restrict__ cu,
                      int32_t* __restrict__ src_idx, uint8_t* __restrict__ keep_out) {
-    extern __shared__ int smem_i[];
-    float* s_score = reinterpret_cast<float*>(smem_i);
-    int* s_kept = smem_i + L_full;
+    extern __shared__ uint64_t smem_k[];
+    const int P = topk_pow2(L_full);
+    uint64_t* s_key = smem_k;
+    int* s_kept = reinterpret_cast<int*>(smem_k + P);
     __shared__ int s_red[kPackThreads / 32];
     const int b = blockIdx.y;
     const int split = blockIdx.x, splits = gridDim.x;
@@ -94,29 +125,45 @@ __global__ void __launch_bounds__(kPackThreads)
     for (int i = tid; i < b; i += kPackThreads) part += clamp_count(__ldg(keep_count + i), L_full);
     part = warp_sum(part);
     if (lane == 0) s_red[warp] = part;
+    const int k = clamp_count(__ldg(keep_count + b), L_full);
+    const int64_t row0 = static_cast<int64_t>(b) * L_full;
+    for (int j = tid; j < P; j += kPackThreads)
+        s_key[j] = (j > 0 && j < L_full) ? topk_key(__ldg(scores + row0 + j), j) : 0ull;
     __syncthreads();
     int base = 0;
 #pragma unroll
     for (int w = 0; w < kPackThreads / 32; ++w) base += s_red[w];
-    const int k = clamp_count(__ldg(keep_count + b), L_full);
-    const int64_t row0 = static_cast<int64_t>(b) * L_full;
-    for (int j = tid; j < L_full; j += kPackThreads) s_score[j] = __ldg(scores + row0 + j);
-    __syncthreads();
 
-    // Token j (> 0) is kept when fewer than k - 1 other non-CLS tokens rank
-    // before it; the survivors are listed in token order (CLS first).
+    // Bitonic sort, descending: in the merge of blocks of `size`, pairs
+    // (lo, lo + stride) are ordered descending where lo & size is 0, else
+    // ascending; the last merge (size = P) is descending throughout.
+    for (int size = 2; size <= P; size <<= 1) {
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+            for (int t = tid; t < P / 2; t += kPackThreads) {
+                const int lo = 2 * t - (t & (stride - 1));
+                const int hi = lo + stride;
+                const uint64_t a = s_key[lo], c = s_key[hi];
+                const bool desc = (lo & size) == 0;
+                if ((a < c) == desc) {
+                    s_key[lo] = c;
+                    s_key[hi] = a;
+                }
+            }
+            __syncthreads();
+        }
+    }
+    // k >= 2: the (k - 1)-th largest non-CLS key; k == 1: nothing beside CLS.
+    const uint64_t cut = k >= 2 ? s_key[k - 2] : ~0ull;
+
+    // Survivors in token order (CLS first).
     int running = 0;
     for (int j0 = 0; j0 < L_full; j0 += kPackThreads) {
         const int j = j0 + tid;
         bool kept = false;
-        if (j == 0) {
+        if (j == 0)
             kept = true;
-        } else if (j < L_full) {
-            const float sj = s_score[j];
-            int before = 0;
-            for (int i = 1; i < L_full && before < k - 1; ++i) before += ranks_before(s_score[i], i, sj, j);
-            kept = before < k - 1;
-        }
+        else if (j < L_full)
+            kept = topk_key(__ldg(scores + row0 + j), j) >= cut;
         if (keep_out != nullptr && split == 0 && j < L_full) keep_out[row0 + j] = kept ? 1 : 0;
         const unsigned bal = __ballot_sync(0xffffffffu, kept);
         __syncthreads();   // s_red of the count above / the previous round is free

@@ -105,8 +105,13 @@ int pack_splits(int64_t B, int64_t L_full) {
 }
 
 bool g_pack_smem[kMaxDevices], g_unpack_smem[kMaxDevices], g_topk_smem[kMaxDevices];
-// Largest L_full of the fused top-k pack: scores and survivor list in shared memory.
+// Largest L_full of the fused top-k pack: sort keys and survivor list in shared memory.
 constexpr int kTopkMaxTokens = 8192;
+// pack_topk_kernel's dynamic shared memory: the padded key array, then the
+// survivor list.
+constexpr int topk_smem_bytes(int L_full) {
+    return ragged::topk_pow2(L_full) * static_cast<int>(sizeof(uint64_t)) + L_full * static_cast<int>(sizeof(int));
+}
 bool g_mma_f16_smem[kMaxDevices], g_mma_bf16_smem[kMaxDevices], g_f32_smem[kMaxDevices];
 
 // Largest dynamic shared memory of the resident kernels: 640 keys and a
@@ -381,9 +386,9 @@ ragged_status ragged_pack_topk(const void* dense, int64_t B, int64_t L_full, int
         return fail(RAGGED_ERR_INVALID_ARG, "dense and packed must be 16-byte aligned");
     if ((reinterpret_cast<uintptr_t>(scores) & 3u) || (reinterpret_cast<uintptr_t>(keep_count) & 3u))
         return fail(RAGGED_ERR_INVALID_ARG, "scores / keep_count must be 4-byte aligned");
-    st = ensure_smem(ragged::pack_topk_kernel, 2 * kTopkMaxTokens * static_cast<int>(sizeof(int)), g_topk_smem);
+    st = ensure_smem(ragged::pack_topk_kernel, topk_smem_bytes(kTopkMaxTokens), g_topk_smem);
     if (st != RAGGED_OK) return st;
-    const int smem = static_cast<int>(2 * L_full * sizeof(int));
+    const int smem = topk_smem_bytes(static_cast<int>(L_full));
     const dim3 grid(pack_splits(B, L_full), static_cast<unsigned>(B));
     ragged::pack_topk_kernel<<<grid, ragged::kPackThreads, smem, s>>>(
         static_cast<const uint4*>(dense), static_cast<int>(L_full), static_cast<uint32_t>(row_bytes / 16), scores,

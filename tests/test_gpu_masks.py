@@ -106,3 +106,39 @@ def test_pack_topk_then_attention():
     T = int(cu_ref[-1])
     got = out[:T].double().cpu().numpy()
     assert np.abs(got - ref).max() <= 4e-3
+
+
+def _special_scores(rng, B, L):
+    """Scores drawn from the values where a sort key could go wrong: both
+    zeros, denormals of both signs, infinities, the extreme finite values and
+    NaNs of several payloads and both signs, mixed with ordinary numbers."""
+    bits = np.array([0x00000000, 0x80000000, 0x00000001, 0x80000001, 0x007fffff, 0x807fffff,
+                     0x7f800000, 0xff800000, 0x7f7fffff, 0xff7fffff, 0x7fc00000, 0xffc00000,
+                     0x7f800001, 0xffffffff, 0x3f800000, 0xbf800000], dtype=np.uint32)
+    pick = bits[rng.integers(0, bits.size, size=(B, L))].view(np.float32)
+    s = np.where(rng.random((B, L)) < 0.6, pick, rng.standard_normal((B, L)).astype(np.float32))
+    return np.ascontiguousarray(s.astype(np.float32))
+
+
+@pytest.mark.parametrize("B,L", [(6, 197), (4, 256), (4, 257), (3, 2), (5, 1), (2, 4097), (2, 8192)])
+def test_pack_topk_special_values(B, L):
+    """Total order on signed zeros (tie), denormals (distinct from zero),
+    infinities and NaN payloads (all tie, below -inf), at lengths on and just
+    past a power of two and at the largest supported length."""
+    rng = synthetic.rng_for(3005, B * 10000 + L)
+    s = _special_scores(rng, B, L)
+    k = rng.integers(1, L + 1, size=B).astype(np.int32)
+    row = 32
+    dense_h = rng.integers(0, 256, size=(B, L, row), dtype=np.uint8)
+    keep_out = torch.full((B, L), 7, dtype=torch.uint8, device="cuda")
+    packed, cu = rv.ragged_pack_topk(torch.from_numpy(dense_h).cuda(), torch.from_numpy(s).cuda(),
+                                     torch.from_numpy(k).cuda(), keep_out=keep_out)
+    torch.cuda.synchronize()
+    keep_ref = oracle.mask_topk(s, k)
+    assert np.array_equal(keep_out.cpu().numpy(), keep_ref)
+    assert np.array_equal(keep_ref.sum(1), k)
+    cu_h = cu.cpu().numpy()
+    assert np.array_equal(cu_h, np.concatenate([[0], np.cumsum(k)]))
+    T = int(cu_h[-1])
+    rows = np.concatenate([dense_h[b][keep_ref[b].astype(bool)] for b in range(B)])
+    assert np.array_equal(packed[:T].cpu().numpy(), rows)

@@ -23,7 +23,8 @@ def _topk_by_lexsort(scores, k):
     B, L = scores.shape
     keep = np.zeros((B, L), dtype=np.uint8)
     for b in range(B):
-        s = scores[b, 1:].astype(np.float64)
+        with np.errstate(invalid="ignore"):                 # signalling NaNs widen quietly
+            s = scores[b, 1:].astype(np.float64)
         nan = np.isnan(s)
         key_score = np.where(nan, 0.0, -s)                 # descending score
         order = np.lexsort((np.arange(1, L), key_score, nan))  # numbers first, then score, then index
@@ -49,6 +50,25 @@ def test_topk_matches_lexsort(ties, nans):
     s = _random_scores(rng, B, L, ties, nans)
     k = rng.integers(-2, L + 5, size=B).astype(np.int32)   # includes out-of-range counts
     assert np.array_equal(oracle.mask_topk(s, k), _topk_by_lexsort(s, k))
+
+
+def test_topk_special_values_match_lexsort():
+    """Signed zeros tie, denormals stay apart from zero, infinities sit at the
+    ends of the numbers, and NaNs of every payload and sign tie below -inf."""
+    bits = np.array([0x00000000, 0x80000000, 0x00000001, 0x80000001, 0x007fffff, 0x807fffff,
+                     0x7f800000, 0xff800000, 0x7f7fffff, 0xff7fffff, 0x7fc00000, 0xffc00000,
+                     0x7f800001, 0xffffffff, 0x3f800000, 0xbf800000], dtype=np.uint32)
+    rng = synthetic.rng_for(2005)
+    B, L = 9, 131
+    s = bits[rng.integers(0, bits.size, size=(B, L))].view(np.float32)
+    k = rng.integers(1, L + 1, size=B).astype(np.int32)
+    assert np.array_equal(oracle.mask_topk(s, k), _topk_by_lexsort(s, k))
+    z = np.array([[0.0, 0.0, -0.0, 0.0]], dtype=np.float32)
+    z[0, 1] = -0.0
+    assert oracle.mask_topk(z, np.array([2])).tolist() == [[1, 1, 0, 0]]   # -0 ties +0: lower index
+    d = np.array([[0.0, 0.0, 0.0, 0.0]], dtype=np.float32)
+    d[0, 3] = np.uint32(1).view(np.float32)                                 # smallest denormal beats zero
+    assert oracle.mask_topk(d, np.array([2])).tolist() == [[1, 0, 0, 1]]
 
 
 def test_topk_closed_cases():
