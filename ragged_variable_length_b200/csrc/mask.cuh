@@ -35,41 +35,34 @@ __device__ __forceinline__ double widen<float>(const void* p, int64_t i) {
 }
 
 constexpr int kMaskThreads = 256;   // 8 tokens per CTA, one warp each
+constexpr int kMaskMaxImages = 65535;   // images per launch (grid y)
 
-constexpr int kMaskBatch = 16;      // loads in flight per lane before they are summed
-
-// keep[t] for the tokens t = 0 .. tokens - 1 (t = b * L_full + j) of x, token t
-// being the C elements from element t * tok_stride.  The sum of squares is
+// keep[b * L_full + j] for the tokens j of the images b = blockIdx.y (one warp
+// per token, blockIdx.x covering 8 tokens of the image); token (b, j) is the C
+// elements from element (b * L_full + j) * tok_stride.  The sum of squares is
 // formed in fp64 in a fixed order, so that the keep decision at the threshold
 // is reproducible: lane l adds the squares of elements l, l + 32, l + 64, ...
 // in turn (every square of an f16, bf16 or f32 element is exact in fp64), then
 // the 32 partial sums are combined pairwise with xor-shuffles 16, 8, 4, 2, 1.
 // Explicit round-to-nearest intrinsics keep the compiler from contracting the
-// multiply-add.  Elements are loaded kMaskBatch at a time before any is
-// added; slots past C load 0, and adding +0 to the (non-negative) sum leaves
-// it unchanged, so the batching does not alter the order's result.
+// multiply-add.
 template <typename T>
 __global__ void __launch_bounds__(kMaskThreads)
-    mask_l2_kernel(const void* __restrict__ x, int64_t tokens, int L_full, int C, int64_t tok_stride, double tau,
+    mask_l2_kernel(const void* __restrict__ x, int L_full, int C, int64_t tok_stride, double tau,
                    uint8_t* __restrict__ keep) {
-    const int64_t t = static_cast<int64_t>(blockIdx.x) * (kMaskThreads / 32) + (threadIdx.x >> 5);
+    const int j = blockIdx.x * (kMaskThreads / 32) + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
-    if (t >= tokens) return;   // warp-uniform
+    if (j >= L_full) return;   // warp-uniform
+    const int64_t t = static_cast<int64_t>(blockIdx.y) * L_full + j;
     const int64_t base = t * tok_stride;
     double ss = 0.0;
-    for (int c0 = 0; c0 < C; c0 += 32 * kMaskBatch) {
-        double v[kMaskBatch];
-#pragma unroll
-        for (int u = 0; u < kMaskBatch; ++u) {
-            const int c = c0 + 32 * u + lane;
-            v[u] = c < C ? widen<T>(x, base + c) : 0.0;
-        }
-#pragma unroll
-        for (int u = 0; u < kMaskBatch; ++u) ss = __dadd_rn(ss, __dmul_rn(v[u], v[u]));
+    for (int c = lane; c < C; c += 32) {
+        const double v = widen<T>(x, base + c);
+        ss = __dadd_rn(ss, __dmul_rn(v, v));
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) ss = __dadd_rn(ss, __shfl_xor_sync(0xffffffffu, ss, off));
-    if (lane == 0) keep[t] = (t % L_full == 0 || __dsqrt_rn(ss) >= tau) ? 1 : 0;
+    if (lane == 0) keep[t] = (j == 0 || __dsqrt_rn(ss) >= tau) ? 1 : 0;
 }
 
 // The top-k order as one unsigned key per token, larger key = ranks earlier:

@@ -353,17 +353,21 @@ ragged_status ragged_mask_l2(const void* x, int64_t B, int64_t L_full, int64_t C
     if (x == nullptr || keep == nullptr) return fail(RAGGED_ERR_INVALID_ARG, "x and keep must not be NULL");
     const int64_t esz = dtype == RAGGED_F32 ? 4 : 2;
     if (reinterpret_cast<uintptr_t>(x) % esz) return fail(RAGGED_ERR_INVALID_ARG, "x is not element-aligned");
-    const int64_t tokens = B * L_full;
-    const unsigned blocks = static_cast<unsigned>((tokens + ragged::kMaskThreads / 32 - 1) / (ragged::kMaskThreads / 32));
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int L = static_cast<int>(L_full), Ci = static_cast<int>(C);
-    if (dtype == RAGGED_F16)
-        ragged::mask_l2_kernel<__half><<<blocks, ragged::kMaskThreads, 0, s>>>(x, tokens, L, Ci, tok_stride, tau, keep);
-    else if (dtype == RAGGED_BF16)
-        ragged::mask_l2_kernel<__nv_bfloat16><<<blocks, ragged::kMaskThreads, 0, s>>>(x, tokens, L, Ci, tok_stride, tau,
-                                                                                      keep);
-    else
-        ragged::mask_l2_kernel<float><<<blocks, ragged::kMaskThreads, 0, s>>>(x, tokens, L, Ci, tok_stride, tau, keep);
+    const unsigned chunks = static_cast<unsigned>((L_full + ragged::kMaskThreads / 32 - 1) / (ragged::kMaskThreads / 32));
+    for (int64_t b0 = 0; b0 < B; b0 += ragged::kMaskMaxImages) {
+        const int64_t nb = B - b0 < ragged::kMaskMaxImages ? B - b0 : ragged::kMaskMaxImages;
+        const dim3 grid(chunks, static_cast<unsigned>(nb));
+        const void* xb = static_cast<const char*>(x) + b0 * L_full * tok_stride * esz;
+        uint8_t* kb = keep + b0 * L_full;
+        if (dtype == RAGGED_F16)
+            ragged::mask_l2_kernel<__half><<<grid, ragged::kMaskThreads, 0, s>>>(xb, L, Ci, tok_stride, tau, kb);
+        else if (dtype == RAGGED_BF16)
+            ragged::mask_l2_kernel<__nv_bfloat16><<<grid, ragged::kMaskThreads, 0, s>>>(xb, L, Ci, tok_stride, tau, kb);
+        else
+            ragged::mask_l2_kernel<float><<<grid, ragged::kMaskThreads, 0, s>>>(xb, L, Ci, tok_stride, tau, kb);
+    }
     return cuda_check(cudaGetLastError(), "mask_l2 launch");
 }
 

@@ -142,3 +142,13 @@ def test_pack_topk_special_values(B, L):
     T = int(cu_h[-1])
     rows = np.concatenate([dense_h[b][keep_ref[b].astype(bool)] for b in range(B)])
     assert np.array_equal(packed[:T].cpu().numpy(), rows)
+
+
+def test_mask_l2_more_images_than_one_launch_holds():
+    """B above the 65,535 images one launch covers: the host splits the batch."""
+    rng = synthetic.rng_for(3006)
+    B, L, C = 70001, 2, 8
+    x = rng.standard_normal((B, L, C)).astype(np.float32)
+    tau = 2.5
+    got = rv.ragged_mask_l2(torch.from_numpy(x).cuda(), tau).cpu().numpy()
+    assert np.array_equal(got, oracle.mask_l2(x, "f32", tau))
