@@ -722,22 +722,31 @@ def deit_block():
     return res
 
 
-def cpu_baseline(min_seconds=10.0):
-    """The CPU oracle, as it stands, on the bench's calls (whole pipeline per call)."""
+def cpu_baseline(min_seconds=10.0, single_thread_seconds=5.0):
+    """The CPU oracle, as it stands, on the bench's calls (whole pipeline per
+    call), on all host cores and, beside it, on one thread."""
     import oracle
     ws = [synthetic.serving(B, p) for B, p in CASES]
-    oracle.pipeline(ws[0])
-    n, t0 = 0, time.perf_counter()
-    while True:
-        for w in ws:
-            oracle.pipeline(w)
-            n += 1
-        if time.perf_counter() - t0 >= min_seconds:
-            break
-    dt = time.perf_counter() - t0
-    return {"value": round(dt * 1e6 / n, 1), "unit": "µs/call", "cores": oracle.num_cores(), "kind": "oracle",
+
+    def timed(seconds, threads):
+        oracle.pipeline(ws[0], threads=threads)
+        n, t0 = 0, time.perf_counter()
+        while True:
+            for w in ws:
+                oracle.pipeline(w, threads=threads)
+                n += 1
+            if time.perf_counter() - t0 >= seconds:
+                break
+        return time.perf_counter() - t0, n
+
+    cores = oracle.num_cores()
+    dt, n = timed(min_seconds, 0)
+    dt1, n1 = timed(single_thread_seconds, 1)
+    return {"value": round(dt * 1e6 / n, 1), "unit": "µs/call", "cores": cores, "kind": "oracle",
             "sample": f"{n} calls ({n // len(ws)} passes over the 12 serving batches), fp64 C oracle, "
-                      f"{oracle.num_cores()} threads"}
+                      f"{cores} threads",
+            "single_thread": {"value": round(dt1 * 1e6 / n1, 1), "unit": "µs/call", "cores": 1,
+                              "sample": f"{n1} calls ({n1 // len(ws)} passes), fp64 C oracle, 1 thread"}}
 
 
 # --------------------------------------------------------------------------
