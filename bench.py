@@ -274,7 +274,7 @@ def run_ours(args, rank, world, dist):
 
     # ---- per-call host / device / total split, per case ----
     detail = {}
-    reps = max(20, min(200, args.steps))
+    reps = args.per_case_calls
     for i, (B, p) in enumerate(CASES):
         host, dev_t, tot = [], [], []
         for r in range(reps):
@@ -293,13 +293,12 @@ def run_ours(args, rank, world, dist):
             t0 = time.perf_counter()
             pl.run_sync()
             tot.append((time.perf_counter() - t0) * 1e6)
-        detail[f"b{B}_p{int(p * 100)}"] = {
-            "host_us": round(statistics.median(host), 2),
-            "device_us": round(statistics.median(dev_t), 2),
-            "total_us": round(statistics.median(tot), 2),
-            "total_p10_us": round(float(np.percentile(tot, 10)), 2),
-            "total_p90_us": round(float(np.percentile(tot, 90)), 2),
-        }
+        entry = {"calls": reps}
+        for name, xs in (("host", host), ("device", dev_t), ("total", tot)):
+            entry[f"{name}_us"] = round(statistics.median(xs), 2)
+            entry[f"{name}_p10_us"] = round(float(np.percentile(xs, 10)), 2)
+            entry[f"{name}_p90_us"] = round(float(np.percentile(xs, 90)), 2)
+        detail[f"b{B}_p{int(p * 100)}"] = entry
 
     # ---- end to end from pinned host buffers ----
     host_in = {}
@@ -830,7 +829,14 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--quick", action="store_true", help="skip the larger workloads and the CPU baseline")
     ap.add_argument("--profile", choices=PROFILE_CASES, help="one untimed pass of a workload (for ncu), no JSON")
+    ap.add_argument("--per-case-calls", type=int, default=None,
+                    help="synchronised calls per (B, rate) for the host/device/total split "
+                         "(default 1000; with --quick, the step count clamped to [20, 200])")
     args = ap.parse_args()
+    if args.per_case_calls is None:
+        args.per_case_calls = max(20, min(200, args.steps)) if args.quick else 1000
+    if args.per_case_calls < 1:
+        ap.error("--per-case-calls must be positive")
     if args.profile:
         run_profile_case(args.profile)
         return
