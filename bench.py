@@ -298,6 +298,14 @@ def run_ours(args, rank, world, dist):
             entry[f"{name}_us"] = round(statistics.median(xs), 2)
             entry[f"{name}_p10_us"] = round(float(np.percentile(xs, 10)), 2)
             entry[f"{name}_p90_us"] = round(float(np.percentile(xs, 90)), 2)
+        # sequences/s from the synchronous total; useful TFLOP/s and the
+        # roofline fraction from the device time of the call
+        w0 = workloads[0][i]
+        dev_s = statistics.median(dev_t) * 1e-6
+        t_roof_case = max(fused_bytes(w0) / (hbm_peak * 1e9), w0.useful_flops() / (bf16_peak * 1e12))
+        entry["seq_per_s"] = round(B / (statistics.median(tot) * 1e-6), 1)
+        entry["useful_tflops"] = round(w0.useful_flops() / dev_s / 1e12, 4)
+        entry["roofline_frac"] = round(t_roof_case / dev_s, 4)
         detail[f"b{B}_p{int(p * 100)}"] = entry
 
     # ---- end to end from pinned host buffers ----
