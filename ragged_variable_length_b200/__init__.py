@@ -11,6 +11,8 @@ Entry points (same names as the C ABI):
   ragged_unpack_cls  CLS row of every sequence
   ragged_unpack      scatter packed rows back to their dense positions
   ragged_pipeline    pack -> attend -> CLS in one host call
+  ragged_mask_l2     Threshold-l2 keep mask from token feature norms
+  ragged_pack_topk   top-k keep selection by score fused into pack
 ``Pipeline`` keeps the buffers and the marshalled arguments of one shape so
 that a call costs one foreign-function crossing, and can replay the whole
 pipeline as one CUDA graph.
