@@ -46,31 +46,36 @@ ragged_status cuda_check(cudaError_t e, const char* what) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Per-device flags and caches may be touched by several host threads at once;
+// the values they hold are idempotent (a second thread repeats the same query
+// or attribute call), so relaxed atomics are enough to make that well defined.
+using DeviceFlags = std::atomic<bool>[kMaxDevices];
+
 // Multiprocessor count of the current device, cached per device.
 int sm_count() {
-    static int cache[kMaxDevices] = {0};
+    static std::atomic<int> cache[kMaxDevices];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
-    if (cache[dev] == 0) {
-        int n = 0;
+    int n = cache[dev].load(std::memory_order_relaxed);
+    if (n == 0) {
         if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
-        cache[dev] = n;
+        cache[dev].store(n, std::memory_order_relaxed);
     }
-    return cache[dev];
+    return n;
 }
 
 // Opt-in shared-memory sizes are set once per device and kernel.
 template <typename Kernel>
-ragged_status ensure_smem(Kernel kernel, int bytes, bool (&done)[kMaxDevices]) {
+ragged_status ensure_smem(Kernel kernel, int bytes, DeviceFlags& done) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
         return fail(RAGGED_ERR_CUDA, "cudaGetDevice failed");
-    if (!done[dev]) {
+    if (!done[dev].load(std::memory_order_relaxed)) {
         ragged_status s = cuda_check(
             cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes),
             "cudaFuncSetAttribute");
         if (s != RAGGED_OK) return s;
-        done[dev] = true;
+        done[dev].store(true, std::memory_order_relaxed);
     }
     return RAGGED_OK;
 }
@@ -104,7 +109,7 @@ int pack_splits(int64_t B, int64_t L_full) {
     return static_cast<int>(s);
 }
 
-bool g_pack_smem[kMaxDevices], g_unpack_smem[kMaxDevices], g_topk_smem[kMaxDevices];
+DeviceFlags g_pack_smem, g_unpack_smem, g_topk_smem;
 // Largest L_full of the fused top-k pack: sort keys and survivor list in shared memory.
 constexpr int kTopkMaxTokens = 8192;
 // pack_topk_kernel's dynamic shared memory: the padded key array, then the
@@ -112,7 +117,7 @@ constexpr int kTopkMaxTokens = 8192;
 constexpr int topk_smem_bytes(int L_full) {
     return ragged::topk_pow2(L_full) * static_cast<int>(sizeof(uint64_t)) + L_full * static_cast<int>(sizeof(int));
 }
-bool g_mma_f16_smem[kMaxDevices], g_mma_bf16_smem[kMaxDevices], g_f32_smem[kMaxDevices];
+DeviceFlags g_mma_f16_smem, g_mma_bf16_smem, g_f32_smem;
 
 // Largest dynamic shared memory of the resident kernels: 640 keys and a
 // 640-entry survivor list.
@@ -132,7 +137,7 @@ int resident_ksplit(int64_t B, int64_t H, int key_tiles) {
 template <typename T, class Src, int KS>
 ragged_status launch_resident_ks(const Src& src, int64_t B, int64_t H, int key_tiles, int list_entries,
                                  float scale, void* out, int64_t out_tok_stride, void* cls_out, void* packed_out,
-                                 bool (&smem_done)[kMaxDevices], cudaStream_t s) {
+                                 DeviceFlags& smem_done, cudaStream_t s) {
     using namespace ragged::resident;
     auto kernel = attn_resident_kernel<T, Src, KS>;
     ragged_status st = ensure_smem(kernel, kResidentSmemMax, smem_done);
@@ -148,7 +153,7 @@ ragged_status launch_resident_ks(const Src& src, int64_t B, int64_t H, int key_t
 }
 
 std::atomic<int> g_attn_kernel{RAGGED_ATTN_AUTO};
-bool g_tc05_smem[2][kMaxDevices];
+DeviceFlags g_tc05_smem[2];
 
 template <typename T>
 ragged_status launch_tc05(const ragged::resident::PackedRows& src, int64_t B, int64_t H, int64_t max_seqlen,
@@ -234,7 +239,7 @@ bool tensor_map_3d(CUtensorMap* out, const void* ptr, int64_t H, int64_t rows, i
     return true;
 }
 
-bool g_persist_smem[2][kMaxDevices];
+DeviceFlags g_persist_smem[2];
 
 // Launches the persistent tcgen05 kernel; *launched = false (and nothing is
 // enqueued) when the launch shape is outside what it supports.
@@ -269,7 +274,7 @@ ragged_status launch_tc05_persist(const ragged::resident::PackedRows& src, int64
 }
 
 // slot: 0/1 packed f16/bf16, 2/3 dense f16/bf16 (one set of smem flags per kernel).
-bool g_res_smem_ks[4][3][kMaxDevices];
+DeviceFlags g_res_smem_ks[4][3];
 
 template <typename T, class Src>
 ragged_status launch_resident(const Src& src, int64_t B, int64_t H, int key_tiles, int list_entries,
