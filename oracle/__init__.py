@@ -40,11 +40,15 @@ _STORAGE = {"f16": np.float16, "bf16": np.uint16, "f32": np.float32, "f64": np.f
 
 
 def build(force: bool = False) -> str:
-    """Compile the oracle with gcc (plain -O2, IEEE semantics) if stale."""
+    """Compile the oracle with gcc (plain -O2, IEEE semantics) if stale.
+
+    -ffp-contract=off (already the ISO C default) is spelled out: no a + b * c
+    may become a fused multiply-add, since the Threshold-l2 sum must round
+    every product and every addition on its own."""
     os.makedirs(os.path.dirname(_LIB), exist_ok=True)
     if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
         tmp = _LIB + f".{os.getpid()}.tmp"
-        subprocess.run(["gcc", "-O2", "-std=c11", "-Wall", "-Wextra", "-shared", "-fPIC",
+        subprocess.run(["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-Wall", "-Wextra", "-shared", "-fPIC",
                         "-pthread", _SRC, "-o", tmp, "-lm"], check=True)
         os.replace(tmp, _LIB)
     return _LIB

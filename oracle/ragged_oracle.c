@@ -28,7 +28,8 @@
  *    first row of every packed sequence;
  *  - scatter-unpack writes kept rows only and leaves dropped rows untouched.
  *
- * Build: gcc -O2 -shared -fPIC -pthread ragged_oracle.c -lm   (no fast-math).
+ * Build: gcc -O2 -std=c11 -ffp-contract=off -shared -fPIC -pthread ragged_oracle.c -lm
+ * (no fast-math, no contraction into fused multiply-adds).
  */
 #include <math.h>
 #include <pthread.h>
