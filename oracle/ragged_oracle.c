@@ -19,7 +19,10 @@
  *    sequences) and the radpulse section "Bypassing the binding" (no causal
  *    mask, no KV cache): for each sequence b and head h,
  *        O = softmax(scale * Q K^T) V   over the L_b rows of sequence b.
- *    The softmax scale 1/sqrt(64) is the usual one; the pages do not print it.
+ *    The softmax scale 1/sqrt(64) is the usual one; the pages do not print it;
+ *  - keep-mask producers (Threshold-l2, score top-k): radpulse article,
+ *    section "Integrated pack pipeline" (the pipeline serves any pruning
+ *    method); their rules are readings, stated where they are defined below.
  *
  * Conventions (readings of the pages where they are silent):
  *  - index 0 (CLS) of every image is kept whatever the mask says;
