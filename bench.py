@@ -789,7 +789,7 @@ def run_reference(args, rank, world):
     }), flush=True)
 
 
-PROFILE_CASES = ("serving", "hires", "sweep")
+PROFILE_CASES = ("serving", "hires", "sweep", "masks")
 
 
 def run_profile_case(case: str) -> None:
@@ -800,6 +800,9 @@ def run_profile_case(case: str) -> None:
              of the streaming mma.sync, tcgen05 and persistent tcgen05 kernels.
     sweep:   the B=512, 0% pruning sweep workload packed, then attention twice
              with each of the same three kernels.
+    masks:   on the B=512, 50% pruning sweep workload: ragged_pack_topk,
+             ragged_mask_l2 over the q features, ragged_pack with the given
+             mask, each launched once.
     """
     import torch
     import ragged_variable_length_b200 as rv
@@ -826,6 +829,20 @@ def run_profile_case(case: str) -> None:
             pl()
             pl()
         rv.ragged_set_attn_kernel(rv.RAGGED_ATTN_AUTO)
+    elif case == "masks":
+        w = synthetic.sweep(0.5)
+        rng = synthetic.rng_for(4001)
+        dense = torch.from_numpy(w.qkv.view(np.int16)).cuda().view(torch.float16)
+        scores = torch.from_numpy(rng.standard_normal((w.B, w.L_full)).astype(np.float32)).cuda()
+        kc = torch.from_numpy(w.lengths.astype(np.int32)).cuda()
+        packed = torch.empty((w.B * w.L_full, 3, w.H, 64), dtype=torch.float16, device="cuda")
+        cu = torch.empty(w.B + 1, dtype=torch.int32, device="cuda")
+        qfeat = dense.view(w.B, w.L_full, 3 * w.H * 64)[:, :, :w.H * 64]
+        keep_given = torch.from_numpy(w.keep).cuda()
+        torch.cuda.synchronize()
+        rv.ragged_pack_topk(dense, scores, kc, packed=packed, cu_seqlens=cu)
+        rv.ragged_mask_l2(qfeat, 8.0)
+        rv.ragged_pack(dense, keep_given, packed=packed, cu_seqlens=cu)
     torch.cuda.synchronize()
 
 
