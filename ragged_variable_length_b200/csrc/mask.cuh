@@ -120,31 +120,57 @@ __global__ void __launch_bounds__(kPackThreads)
     if (lane == 0) s_red[warp] = part;
     const int k = clamp_count(__ldg(keep_count + b), L_full);
     const int64_t row0 = static_cast<int64_t>(b) * L_full;
-    for (int j = tid; j < P; j += kPackThreads)
-        s_key[j] = (j > 0 && j < L_full) ? topk_key(__ldg(scores + row0 + j), j) : 0ull;
-    __syncthreads();
-    int base = 0;
-#pragma unroll
-    for (int w = 0; w < kPackThreads / 32; ++w) base += s_red[w];
 
     // Bitonic sort, descending: in the merge of blocks of `size`, pairs
     // (lo, lo + stride) are ordered descending where lo & size is 0, else
     // ascending; the last merge (size = P) is descending throughout.
-    for (int size = 2; size <= P; size <<= 1) {
-        for (int stride = size >> 1; stride > 0; stride >>= 1) {
-            for (int t = tid; t < P / 2; t += kPackThreads) {
-                const int lo = 2 * t - (t & (stride - 1));
-                const int hi = lo + stride;
-                const uint64_t a = s_key[lo], c = s_key[hi];
-                const bool desc = (lo & size) == 0;
-                if ((a < c) == desc) {
-                    s_key[lo] = c;
-                    s_key[hi] = a;
+    if (P <= kPackThreads) {
+        // One key per thread (slot tid).  A slot's partner is tid ^ stride, in
+        // the same block of `size` <= P, so slots below P only ever meet
+        // slots below P; the slots from P up hold keys nobody reads.  Strides
+        // below 32 pair lanes of one warp (a shuffle, no barrier); the others
+        // exchange through shared memory.
+        uint64_t key = (tid > 0 && tid < L_full) ? topk_key(__ldg(scores + row0 + tid), tid) : 0ull;
+        for (int size = 2; size <= P; size <<= 1) {
+            for (int stride = size >> 1; stride > 0; stride >>= 1) {
+                uint64_t other;
+                if (stride >= 32) {
+                    if (tid < P) s_key[tid] = key;
+                    __syncthreads();
+                    other = tid < P ? s_key[tid ^ stride] : key;
+                    __syncthreads();
+                } else {
+                    other = __shfl_xor_sync(0xffffffffu, key, stride);
                 }
+                const bool desc = (tid & size) == 0, lower = (tid & stride) == 0;
+                key = (lower == desc) ? (key > other ? key : other) : (key < other ? key : other);
             }
-            __syncthreads();
+        }
+        if (tid < P) s_key[tid] = key;
+        __syncthreads();
+    } else {
+        for (int j = tid; j < P; j += kPackThreads)
+            s_key[j] = (j > 0 && j < L_full) ? topk_key(__ldg(scores + row0 + j), j) : 0ull;
+        __syncthreads();
+        for (int size = 2; size <= P; size <<= 1) {
+            for (int stride = size >> 1; stride > 0; stride >>= 1) {
+                for (int t = tid; t < P / 2; t += kPackThreads) {
+                    const int lo = 2 * t - (t & (stride - 1));
+                    const int hi = lo + stride;
+                    const uint64_t a = s_key[lo], c = s_key[hi];
+                    const bool desc = (lo & size) == 0;
+                    if ((a < c) == desc) {
+                        s_key[lo] = c;
+                        s_key[hi] = a;
+                    }
+                }
+                __syncthreads();
+            }
         }
     }
+    int base = 0;
+#pragma unroll
+    for (int w = 0; w < kPackThreads / 32; ++w) base += s_red[w];
     // k >= 2: the (k - 1)-th largest non-CLS key; k == 1: nothing beside CLS.
     const uint64_t cut = k >= 2 ? s_key[k - 2] : ~0ull;
 
