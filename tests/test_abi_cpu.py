@@ -206,6 +206,8 @@ def test_device_status_needs_an_output_pointer(lib):
     assert lib.ragged_get_device_status(None, None) == rv.RAGGED_ERR_INVALID_ARG
 
 
-def test_binding_fails_loudly_without_the_library(tmp_path):
+def test_binding_fails_loudly_without_the_library():
+    missing = os.path.join(os.path.dirname(os.path.abspath(__file__)), "no_such_dir", "nope.so")
+    assert not os.path.exists(missing)
     with pytest.raises(RuntimeError, match="missing"):
-        rv.load(str(tmp_path / "nope.so"))
+        rv.load(missing)

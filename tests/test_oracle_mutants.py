@@ -68,15 +68,21 @@ def source():
     return open(SRC).read()
 
 
+# Mutant copies are built beside the oracle's own library (a git-ignored folder).
+MUTANT_DIR = os.path.join(os.path.dirname(SRC), "_build", "mutants")
+
+
 @pytest.mark.parametrize("name", sorted(MUTANTS))
-def test_pins_catch_mutant(name, source, tmp_path):
+def test_pins_catch_mutant(name, source):
     old, new = MUTANTS[name]
     assert source.count(old) == 1, f"mutation site for {name} not found exactly once"
-    mutant_src = tmp_path / f"{name}.c"
-    mutant_src.write_text(source.replace(old, new))
-    so = tmp_path / f"lib{name}.so"
-    subprocess.run(["gcc", "-O2", "-std=c11", "-shared", "-fPIC", "-pthread", str(mutant_src),
-                    "-o", str(so), "-lm"], check=True)
+    os.makedirs(MUTANT_DIR, exist_ok=True)
+    mutant_src = os.path.join(MUTANT_DIR, f"{name}.c")
+    with open(mutant_src, "w") as f:
+        f.write(source.replace(old, new))
+    so = os.path.join(MUTANT_DIR, f"lib{name}.so")
+    subprocess.run(["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-shared", "-fPIC", "-pthread", mutant_src,
+                    "-o", so, "-lm"], check=True)
     real = oracle._load()
     oracle.use_library(oracle.bind(str(so)))
     caught = 0
