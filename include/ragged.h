@@ -177,7 +177,10 @@ RAGGED_API int32_t ragged_set_attn_kernel(int32_t kernel);
  *   x           device, token (b, j) is the C elements starting at element
  *               (b * L_full + j) * tok_stride; f16, bf16 or f32 (dtype),
  *               aligned to its element size.  Read only.
- *   B, L_full   as for ragged_pack (B * L_full < 2^31).
+ *   B, L_full   B >= 0 images (B = 0 is a no-op), 1 <= L_full <= RAGGED_MAX_TOKENS,
+ *               B * L_full < 2^31 (else RAGGED_ERR_UNSUPPORTED).  One launch
+ *               covers up to 65,535 images; larger batches take several,
+ *               enqueued in order on the stream.
  *   C           elements per token, 1 <= C <= 2^24; tok_stride >= C.
  *   tau         threshold, not NaN; tau <= 0 keeps every token.
  *   keep        device uint8 [B, L_full]: 1 kept, 0 dropped (an input for
