@@ -79,8 +79,8 @@ typedef enum ragged_dtype {
  *
  *   dense       device, [B, L_full] rows of row_bytes bytes, contiguous,
  *               16-byte aligned.  Read only.
- *   B, L_full   images and dense tokens per image; B >= 0, 1 <= L_full <=
- *               RAGGED_MAX_TOKENS.
+ *   B, L_full   images and dense tokens per image; 0 <= B <= 65535 (above:
+ *               RAGGED_ERR_UNSUPPORTED), 1 <= L_full <= RAGGED_MAX_TOKENS.
  *   row_bytes   bytes per token row; a positive multiple of 16.
  *   keep        device, uint8 [B, L_full], any alignment.  Nonzero keeps the
  *               token.  Token 0 (CLS) is kept whatever keep[b, 0] says.
@@ -117,7 +117,8 @@ RAGGED_API ragged_status ragged_pack(const void *dense, int64_t B, int64_t L_ful
  *                  be a multiple of 16 bytes.
  *   cu_seqlens     device int32 [B + 1], non-decreasing, cu[0] = 0 (as
  *                  written by ragged_pack).  Read on the device only.
- *   B              number of sequences, >= 0 (0 is a no-op).
+ *   B              number of sequences, 0 .. 65535 (0 is a no-op; above:
+ *                  RAGGED_ERR_UNSUPPORTED).
  *   max_seqlen     host-side upper bound on every L_b (e.g. L_full), 1 ..
  *                  RAGGED_MAX_TOKENS.  Sizes the launch; a sequence longer
  *                  than this is skipped and RAGGED_DEV_BAD_SEQLENS is set.
@@ -238,6 +239,7 @@ RAGGED_API ragged_status ragged_unpack_cls(const void *packed, const int32_t *cu
  *   cu_seqlens  device int32 [B + 1] from ragged_pack on the same keep mask.
  *   keep        device uint8 [B, L_full].
  *   dense_out   device [B, L_full] rows of row_bytes, 16-byte aligned.
+ *   B, L_full, row_bytes   limits as for ragged_pack.
  */
 RAGGED_API ragged_status ragged_unpack(const void *packed, const int32_t *cu_seqlens, const uint8_t *keep,
                             int64_t B, int64_t L_full, int64_t row_bytes, void *dense_out,
