@@ -167,8 +167,9 @@ def tiny(dtype: str = "f16", seed: int = 1001) -> Workload:
 
     tokens [4,197,384] float32 N(0,1); W_q, W_k, W_v float32 N(0, 1/384),
     head h = output columns 64h..64h+63.  The projection is a model layer
-    outside the pipeline; it is applied here, on the host, in float64 and
-    rounded once to ``dtype``.  It acts row by row, so it commutes with packing.
+    outside the pipeline; it is applied here, on the host, in float64, rounded
+    to float32 (the tokens' format) and then stored in ``dtype``.  It acts row
+    by row, so it commutes with packing.
     """
     rng = rng_for(seed, 0)
     B, L_full, C, H, d = 4, 197, 384, 6, 64
