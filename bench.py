@@ -193,6 +193,18 @@ def pack_bytes(w) -> int:
     return w.B * w.L_full + 2 * w.T * w.row_bytes + 4 * (w.B + 1)
 
 
+def optional(fn):
+    """Runs one of the extra measurements.  A Python-level failure there is
+    reported in its key (and its traceback on stderr) instead of ending the
+    run before the JSON line with the headline number is printed."""
+    try:
+        return fn()
+    except Exception as e:  # noqa: BLE001 - any failure of an extra is reported, not raised
+        import traceback
+        traceback.print_exc()
+        return {"error": f"{type(e).__name__}: {e}"[:300]}
+
+
 def run_ours(args, rank, world, dist):
     import torch
     import ragged_variable_length_b200 as rv
@@ -417,8 +429,8 @@ def run_ours(args, rank, world, dist):
                                "pack_GBps": round(b_pack / t_pack / 1e9, 2)}}
 
     # ---- larger workloads: attention roofline (single GPU, same kernel family) ----
-    larger = {}
-    if not args.quick and world == 1:
+    def measure_larger():
+        larger = {}
         for name, make, copies in (("deit_b_p80_b32", lambda c: synthetic.make_workload(
                                         "deit_b_p80_b32", 32, 197, 12,
                                         synthetic.deit_b_pruned80().lengths, "bf16", 1002, 1 + c), 36),
@@ -455,19 +467,21 @@ def run_ours(args, rank, world, dist):
                             "l2": f"inputs rotated over {copies} copies" if copies > 1 else "packed q/k/v exceed L2"}
             del pls
             torch.cuda.empty_cache()
+        return larger
+
+    single = world == 1 and not args.quick
+    larger = optional(measure_larger) if single else {}
 
     # ---- padded PyTorch SDPA baseline, same calls, same synchronisation ----
-    padded = padded_baseline(args, pipes, workloads, ncopies, stream)
+    padded = optional(lambda: padded_baseline(args, pipes, workloads, ncopies, stream))
 
     # ---- other attention paths on the same calls, and the mask producers ----
-    comps = comparators(args, pipes, workloads, stream) if world == 1 and not args.quick else None
-    masks = mask_producers() if world == 1 and not args.quick else None
-    block = deit_block() if world == 1 and not args.quick else None
+    comps = optional(lambda: comparators(args, pipes, workloads, stream)) if single else None
+    masks = optional(mask_producers) if single else None
+    block = optional(deit_block) if single else None
 
     # ---- CPU oracle on a bounded sample (rank 0, one GPU only) ----
-    cpu = None
-    if rank == 0 and world == 1 and not args.quick:
-        cpu = cpu_baseline(min_seconds=10.0)
+    cpu = optional(lambda: cpu_baseline(min_seconds=10.0)) if rank == 0 and single else None
 
     gpu_launches = 1 * args.steps * len(CASES)   # one fused launch per call
     hw = {"metric": "ragged attn µs/call (host+device) at BS1-4; useful TFLOP/s & % roofline",

@@ -112,3 +112,13 @@ def test_recorded_traffic_is_withheld_when_sources_change(monkeypatch):
 def test_committed_traffic_record_matches_the_current_kernel():
     """The committed DRAM record belongs to the fused kernel as it stands."""
     assert bench.recorded_traffic() is not None
+
+
+def test_a_failing_extra_measurement_is_reported_not_raised(capsys):
+    """The JSON line must survive a failure in one of the optional measurements."""
+    def boom():
+        raise RuntimeError("comparator unavailable")
+    assert bench.optional(lambda: {"x": 1}) == {"x": 1}
+    rec = bench.optional(boom)
+    assert rec == {"error": "RuntimeError: comparator unavailable"}
+    assert "comparator unavailable" in capsys.readouterr().err
