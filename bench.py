@@ -513,13 +513,27 @@ def run_ours(args, rank, world, dist):
         print(json.dumps(hw), flush=True)
 
 
+def sdpa_backend(q, k, v, mask) -> str:
+    """Name of the SDPA backend torch's dispatcher picks for these arguments
+    (torch._fused_sdp_choice, mapped through the public SDPBackend enum)."""
+    try:
+        import torch
+        from torch.nn.attention import SDPBackend
+        names = {int(b): n for n, b in SDPBackend.__members__.items()}
+        return names.get(int(torch._fused_sdp_choice(q, k, v, mask, 0.0, False)), "unknown")
+    except Exception as e:  # noqa: BLE001 - a private query; its failure is only reported
+        return f"unknown ({type(e).__name__})"
+
+
 def padded_baseline(args, pipes, workloads, ncopies, stream):
     """Pad every survivor set to the batch's longest (Lmax known on the host),
-    mask padded keys, run torch SDPA, take the CLS rows."""
+    mask padded keys, run torch SDPA, take the CLS rows.  Each case records
+    the SDPA backend that runs."""
     import torch
     import torch.nn.functional as F
+    backends = {}
 
-    def call(pl, Lmax):
+    def call(pl, Lmax, probe=False):
         keep = pl.keep.bool()
         keep[:, 0] = True
         L = keep.sum(1)
@@ -528,6 +542,8 @@ def padded_baseline(args, pipes, workloads, ncopies, stream):
         g = torch.gather(pl.dense_qkv, 1, idx[:, :, None, None, None].expand(B, Lmax, three, H, d))
         q, k, v = g.permute(2, 0, 3, 1, 4).unbind(0)             # [B, H, Lmax, d]
         valid = torch.arange(Lmax, device=keep.device)[None, :] < L[:, None]
+        if probe:   # outside the timed calls
+            backends[(B, Lmax)] = sdpa_backend(q, k, v, valid[:, None, None, :])
         o = F.scaled_dot_product_attention(q, k, v, attn_mask=valid[:, None, None, :])
         return o[:, :, 0]
 
@@ -545,8 +561,9 @@ def padded_baseline(args, pipes, workloads, ncopies, stream):
             if r >= 3:
                 tot.append((time.perf_counter() - t0) * 1e6)
         ref = pipes[0][i].cls_out.float()
-        err = float((call(pipes[0][i], int(workloads[0][i].Lmax)).float() - ref).abs().max())
-        res[f"b{B}_p{int(p * 100)}"] = {"total_us": round(statistics.median(tot), 2), "max_abs_vs_ragged": err}
+        err = float((call(pipes[0][i], int(workloads[0][i].Lmax), probe=True).float() - ref).abs().max())
+        res[f"b{B}_p{int(p * 100)}"] = {"total_us": round(statistics.median(tot), 2), "max_abs_vs_ragged": err,
+                                         "sdpa_backend": backends.get((B, int(workloads[0][i].Lmax)), "unknown")}
     return res
 
 

@@ -122,3 +122,13 @@ def test_a_failing_extra_measurement_is_reported_not_raised(capsys):
     rec = bench.optional(boom)
     assert rec == {"error": "RuntimeError: comparator unavailable"}
     assert "comparator unavailable" in capsys.readouterr().err
+
+
+def test_sdpa_backend_is_named():
+    """The padded baseline names the SDPA backend torch picks for its call."""
+    import torch
+    from torch.nn.attention import SDPBackend
+    q = torch.randn(2, 3, 5, 64)
+    mask = torch.ones(2, 1, 1, 5, dtype=torch.bool)
+    name = bench.sdpa_backend(q, q, q, mask)
+    assert name in SDPBackend.__members__ or name.startswith("unknown")
