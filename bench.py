@@ -291,13 +291,14 @@ def run_ours(args, rank, world, dist):
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
-    h0, h1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    h0.record(stream)
+    warm_start, warm_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    warm_start.record(stream)
     for _ in range(args.steps):
         step(0)
-    h1.record(stream)
+    warm_end.record(stream)
     torch.cuda.synchronize()
-    warm_us = us_per_call(max_over_ranks(h0.elapsed_time(h1), dist, dev), args.steps, len(CASES), world)
+    warm_ms = max_over_ranks(warm_start.elapsed_time(warm_end), dist, dev)
+    warm_us = us_per_call(warm_ms, args.steps, len(CASES), world)
 
     # ---- per-call host / device / total split, per case ----
     detail = {}
