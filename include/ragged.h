@@ -284,6 +284,50 @@ RAGGED_API ragged_status ragged_pipeline(const void *dense_qkv, const uint8_t *k
                                          ragged_dtype dtype, void *packed_qkv, int32_t *cu_seqlens,
                                          void *out, void *cls_out, uint32_t flags, void *stream);
 
+/* Bytes of the fixed device scratch behind ragged_pipeline_noalloc (16 MiB). */
+#define RAGGED_NOALLOC_SCRATCH_BYTES (16ll << 20)
+
+/*
+ * ragged_pipeline_noalloc - ragged_pipeline in its two-launch form, for
+ * callers that must not allocate device memory.  The paper has no
+ * counterpart: it is a packaging of the same pack and attention launches.
+ *
+ * Who needs it: a plugin hosted by a framework or inference server whose own
+ * allocator owns all of device memory (a cudaMalloc behind its back breaks
+ * its accounting or fails), code that runs while some thread captures a CUDA
+ * graph in global capture mode (cudaMalloc is then an error), and services
+ * that fix their device footprint when they start.  Such a caller can still
+ * hand in its inputs and outputs, but not the packed q/k/v that the
+ * two-launch pipeline passes from pack to attention.
+ *
+ * Here that intermediate lives in a fixed array of RAGGED_NOALLOC_SCRATCH_BYTES
+ * bytes inside the library's device image.  Every GPU on which the library's
+ * kernels are loaded holds it until the process exits.  The call allocates
+ * nothing: no cudaMalloc, no cudaFree, no allocating library routine.
+ *
+ *   Arguments as ragged_pipeline, without packed_qkv and flags: dense_qkv
+ *   [B, L_full, 3, H, head_dim], keep, cu_seqlens [B + 1], out (capacity
+ *   B * L_full rows, token stride H * head_dim), cls_out (or NULL), stream.
+ *   Results are identical to ragged_pipeline with RAGGED_PIPELINE_SPLIT.
+ *
+ * Limit: B * L_full * 3 * H * head_dim * element size must not exceed
+ * RAGGED_NOALLOC_SCRATCH_BYTES (every token may survive); larger requests
+ * return RAGGED_ERR_UNSUPPORTED before anything is enqueued.
+ *
+ * The first call on a device looks up the array's device address for that
+ * device (cudaGetSymbolAddress, with that device current) and caches it; make
+ * that first call before any stream capture.  All calls share the one array
+ * and it keeps what the last call left there; nothing in it needs to start at
+ * zero, since pack writes every row that attention then reads.  Two calls
+ * whose work overlaps on the GPU (different streams, or different host
+ * threads, without ordering between them) race on the array and may return
+ * wrong results: order them on one stream or with events.
+ */
+RAGGED_API ragged_status ragged_pipeline_noalloc(const void *dense_qkv, const uint8_t *keep, int64_t B,
+                                                 int64_t L_full, int64_t H, int64_t head_dim, float scale,
+                                                 ragged_dtype dtype, int32_t *cu_seqlens, void *out,
+                                                 void *cls_out, void *stream);
+
 /*
  * ragged_get_device_status - read and clear the status word of the current
  * device.  Synchronises with `stream` (the only call that does).  *host_out

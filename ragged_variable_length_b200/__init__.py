@@ -13,6 +13,8 @@ Entry points (same names as the C ABI):
   ragged_pipeline    pack -> attend -> CLS in one host call
   ragged_mask_l2     Threshold-l2 keep mask from token feature norms
   ragged_pack_topk   top-k keep selection by score fused into pack
+  ragged_pipeline_noalloc  the two-launch pipeline with its packed q/k/v in a
+                     fixed library array, for callers that cannot allocate
 ``Pipeline`` keeps the buffers and the marshalled arguments of one shape so
 that a call costs one foreign-function crossing, and can replay the whole
 pipeline as one CUDA graph.
@@ -36,6 +38,7 @@ RAGGED_ERR_DEVICE = 4
 RAGGED_DEV_BAD_SEQLENS = 0x1
 RAGGED_DEV_TIMEOUT = 0x2
 RAGGED_MAX_TOKENS = 16384
+RAGGED_NOALLOC_SCRATCH_BYTES = 16 << 20
 RAGGED_PIPELINE_AUTO = 0
 RAGGED_PIPELINE_FUSED = 1
 RAGGED_PIPELINE_SPLIT = 2
@@ -53,7 +56,7 @@ DTYPE_NAMES = {"f16": torch.float16, "bf16": torch.bfloat16, "f32": torch.float3
 EXPORTS = ("ragged_pack", "ragged_attn_fwd", "ragged_unpack_cls", "ragged_unpack",
            "ragged_pipeline", "ragged_get_device_status", "ragged_status_string",
            "ragged_last_error", "ragged_abi_version", "ragged_set_attn_kernel",
-           "ragged_mask_l2", "ragged_pack_topk")
+           "ragged_mask_l2", "ragged_pack_topk", "ragged_pipeline_noalloc")
 
 
 class RaggedError(RuntimeError):
@@ -82,9 +85,10 @@ def load(path: Optional[str] = None):
     lib.ragged_pack_topk.argtypes = [vp, i64, i64, i64, vp, vp, vp, vp, vp, vp, vp]
     lib.ragged_unpack.argtypes = [vp, vp, vp, i64, i64, i64, vp, vp]
     lib.ragged_pipeline.argtypes = [vp, vp, i64, i64, i64, i64, f32, i32, vp, vp, vp, vp, ctypes.c_uint32, vp]
+    lib.ragged_pipeline_noalloc.argtypes = [vp, vp, i64, i64, i64, i64, f32, i32, vp, vp, vp, vp]
     lib.ragged_get_device_status.argtypes = [ctypes.POINTER(ctypes.c_uint32), vp]
     for name in ("ragged_pack", "ragged_attn_fwd", "ragged_unpack_cls", "ragged_unpack",
-                 "ragged_pipeline", "ragged_get_device_status"):
+                 "ragged_pipeline", "ragged_get_device_status", "ragged_pipeline_noalloc"):
         getattr(lib, name).restype = ctypes.c_int
     lib.ragged_status_string.argtypes = [ctypes.c_int]
     lib.ragged_status_string.restype = ctypes.c_char_p
@@ -272,6 +276,26 @@ def ragged_pipeline(dense_qkv: torch.Tensor, keep: torch.Tensor, scale: Optional
                                   _dtype_code(dense_qkv), _ptr(packed_qkv), _ptr(cu_seqlens), _ptr(out),
                                   _ptr(cls_out), int(flags), _stream(stream)))
     return packed_qkv, cu_seqlens, out, cls_out
+
+
+def ragged_pipeline_noalloc(dense_qkv: torch.Tensor, keep: torch.Tensor, cu_seqlens: torch.Tensor,
+                            out: torch.Tensor, cls_out: Optional[torch.Tensor] = None,
+                            scale: Optional[float] = None, stream=None):
+    """ragged_pipeline's two-launch form with the packed q/k/v in the library's
+    fixed device array: allocates nothing, so every output is passed in.
+
+    dense_qkv [B, L_full, 3, H, 64]; cu_seqlens int32 [B + 1]; out [B * L_full, H, 64];
+    cls_out [B, H, 64] or None.  B * L_full * 3 * H * 64 * element size must not
+    exceed RAGGED_NOALLOC_SCRATCH_BYTES.  Calls that overlap on the GPU race on
+    the shared array.
+    """
+    B, L_full, three, H, d = dense_qkv.shape
+    if scale is None:
+        scale = d ** -0.5
+    _check(load().ragged_pipeline_noalloc(_ptr(dense_qkv), _ptr(keep), B, L_full, H, d, float(scale),
+                                          _dtype_code(dense_qkv), _ptr(cu_seqlens), _ptr(out), _ptr(cls_out),
+                                          _stream(stream)))
+    return cu_seqlens, out, cls_out
 
 
 def ragged_get_device_status(stream=None) -> int:

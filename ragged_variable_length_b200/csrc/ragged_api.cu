@@ -293,6 +293,40 @@ ragged_status launch_resident(const Src& src, int64_t B, int64_t H, int key_tile
     }
 }
 
+// ---- fixed scratch of ragged_pipeline_noalloc ---------------------------------
+//
+// The packed q/k/v between the pack and the attention launch, for callers that
+// cannot allocate device memory.  It is part of this library's device image:
+// every GPU on which the library's kernels are loaded holds these bytes until
+// the process exits, whether or not the entry point is ever called.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[RAGGED_NOALLOC_SCRATCH_BYTES];
+
+// Device address of g_noalloc_scratch, looked up once per device.  In host
+// code the array's name only stands in for the symbol; the address a kernel
+// may use comes from cudaGetSymbolAddress with that device current.
+std::atomic<void*> g_noalloc_addr[kMaxDevices];
+std::mutex g_noalloc_mu;
+
+ragged_status noalloc_scratch(void** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+        return fail(RAGGED_ERR_CUDA, "cudaGetDevice failed");
+    void* p = g_noalloc_addr[dev].load(std::memory_order_acquire);
+    if (p == nullptr) {
+        std::lock_guard<std::mutex> lock(g_noalloc_mu);
+        p = g_noalloc_addr[dev].load(std::memory_order_relaxed);
+        if (p == nullptr) {
+            ragged_status st = cuda_check(cudaGetSymbolAddress(&p, g_noalloc_scratch),
+                                          "cudaGetSymbolAddress of the fixed scratch");
+            if (st != RAGGED_OK) return st;
+            if (p == nullptr) return fail(RAGGED_ERR_CUDA, "cudaGetSymbolAddress returned NULL");
+            g_noalloc_addr[dev].store(p, std::memory_order_release);
+        }
+    }
+    *out = p;
+    return RAGGED_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -633,5 +667,28 @@ ragged_status ragged_get_device_status(uint32_t* host_out, void* stream) {
     *host_out = value;
     return RAGGED_OK;
 }
+
+ragged_status ragged_pipeline_noalloc(const void* dense_qkv, const uint8_t* keep, int64_t B, int64_t L_full,
+                                      int64_t H, int64_t head_dim, float scale, ragged_dtype dtype,
+                                      int32_t* cu_seqlens, void* out, void* cls_out, void* stream) {
+    if (head_dim != 64) return fail(RAGGED_ERR_UNSUPPORTED, "head_dim = %lld (only 64 is implemented)", (long long)head_dim);
+    if (H < 1 || H > 65535) return fail(RAGGED_ERR_INVALID_ARG, "H = %lld outside [1, 65535]", (long long)H);
+    if (dtype != RAGGED_F16 && dtype != RAGGED_BF16 && dtype != RAGGED_F32)
+        return fail(RAGGED_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
+    const int64_t row_bytes = 3 * H * head_dim * (dtype == RAGGED_F32 ? 4 : 2);
+    ragged_status st = check_rows(B, L_full, row_bytes);
+    if (st != RAGGED_OK) return st;
+    // Every one of the B * L_full rows may survive, so that is what must fit.
+    if (B * L_full > static_cast<int64_t>(RAGGED_NOALLOC_SCRATCH_BYTES) / row_bytes)
+        return fail(RAGGED_ERR_UNSUPPORTED,
+                    "B * L_full * row_bytes = %lld bytes of packed q/k/v exceed the fixed scratch of %lld bytes",
+                    (long long)(B * L_full * row_bytes), (long long)RAGGED_NOALLOC_SCRATCH_BYTES);
+    void* scratch = nullptr;
+    st = noalloc_scratch(&scratch);
+    if (st != RAGGED_OK) return st;
+    return ragged_pipeline(dense_qkv, keep, B, L_full, H, head_dim, scale, dtype, scratch, cu_seqlens, out,
+                           cls_out, RAGGED_PIPELINE_SPLIT, stream);
+}
+
 
 }  // extern "C"
