@@ -183,13 +183,16 @@ RAGGED_API int32_t ragged_set_attn_kernel(int32_t kernel);
  *               covers up to 65,535 images; larger batches take several,
  *               enqueued in order on the stream.
  *   C           elements per token, 1 <= C <= 2^24; tok_stride >= C.
- *   tau         threshold, not NaN; tau <= 0 keeps every token.
+ *   tau         threshold, not NaN.
  *   keep        device uint8 [B, L_full]: 1 kept, 0 dropped (an input for
  *               ragged_pack / ragged_pipeline).
- * The sum of squares is formed in fp64 in a fixed order (lane l of a warp sums
- * the squares of elements l, l + 32, ..., then the 32 partials are combined
- * pairwise: 16, 8, 4, 2, 1) and compared as a correctly rounded square root,
- * so the decision is reproducible bit for bit.
+ * The decision is exact, whatever the order of summation: a token is kept
+ * when sum(x_c^2) >= tau^2 in exact arithmetic, CLS always.  With tau <= 0
+ * every token is kept except those with a NaN element, which are always
+ * dropped; a token with an infinite element (and no NaN) is always kept.  An
+ * fp64 sum settles the bit unless it lies within a relative 2^-26 of tau^2;
+ * there one lane forms the sum exactly, as an integer multiple of 2^-298,
+ * which costs O(C) serial steps for that token.
  */
 RAGGED_API ragged_status ragged_mask_l2(const void *x, int64_t B, int64_t L_full, int64_t C, int64_t tok_stride,
                                         ragged_dtype dtype, double tau, uint8_t *keep, void *stream);
@@ -231,7 +234,10 @@ RAGGED_API ragged_status ragged_unpack_cls(const void *packed, const int32_t *cu
 
 /*
  * ragged_unpack - scatter back (step 3, full form).
- * The inverse of ragged_pack's gather: dense_out[b, j] = packed[cu[b] + r]
+ * Paper: the pipeline's last step, "scatter the result back, or extract the
+ * CLS rows" (the pack-attend-unpack pipeline of the abstract), and radpulse
+ * section "Integrated pack pipeline" (survivors kept in a flat tensor whose
+ * rows map back to their images).  The inverse of ragged_pack's gather: dense_out[b, j] = packed[cu[b] + r]
  * for the r-th survivor j of image b (same keep mask, CLS always kept).  Rows
  * of dropped tokens are left untouched.
  *

@@ -18,6 +18,11 @@ Vision Transformers"):
   mask_topk / mask_l2 keep-mask producers (radpulse "Integrated pack
                       pipeline": the pipeline serves any pruning method, e.g.
                       Threshold-l2); the rules are readings, see the C file
+  deit_block_cls      one encoder block on each image's survivors, CLS rows
+                      out (radpulse "Integrated pack pipeline": attention and
+                      the MLP run on the packed tokens, then CLS is
+                      extracted; "Implications": the MLP acts token by token);
+                      plain numpy float64
 """
 from __future__ import annotations
 
@@ -230,3 +235,50 @@ def mask_l2(x: np.ndarray, dtype: str, tau: float) -> np.ndarray:
     keep = np.zeros((B, L_full), dtype=np.uint8)
     _load().oracle_mask_l2(_ptr(x), DTYPE_CODES[dtype], B, L_full, C, C, float(tau), _ptr(keep))
     return keep
+
+
+def deit_block_cls(x: np.ndarray, keep: np.ndarray, Wqkv: np.ndarray, Wo: np.ndarray, W1: np.ndarray,
+                   W2: np.ndarray, H: int, scale: float = 0.125, eps: float = 1e-5) -> np.ndarray:
+    """CLS row of one pre-norm transformer encoder block applied to each
+    image's surviving tokens, in float64.
+
+    x [B, L_full, D] and the weights are float arrays (widened exactly); keep
+    uint8 [B, L_full], token 0 always kept.  Linears carry no bias and the
+    layer norms no affine parameters (unit weights, zero biases), so for the
+    tokens t of one image:
+        h = t + Attn(LN(t)) Wo^T,          Attn per head over the image's own tokens:
+                                           softmax(scale q k^T) v, with [q k v] = LN(t) Wqkv^T
+        y = h + GELU(LN(h) W1^T) W2^T,     GELU(z) = z (1 + erf(z / sqrt 2)) / 2
+    LN(z) = (z - mean) / sqrt(var + eps), var the biased variance over D.
+    Returns y[CLS] for every image, [B, D] float64.
+    """
+    from math import erf, sqrt
+    x = np.asarray(x, dtype=np.float64)
+    Wqkv, Wo, W1, W2 = (np.asarray(w, dtype=np.float64) for w in (Wqkv, Wo, W1, W2))
+    B, L_full, D = x.shape
+    d = D // H
+    erf_v = np.vectorize(erf)
+
+    def layer_norm(z):
+        mu = z.mean(axis=1, keepdims=True)
+        var = ((z - mu) ** 2).mean(axis=1, keepdims=True)
+        return (z - mu) / np.sqrt(var + eps)
+
+    out = np.zeros((B, D), dtype=np.float64)
+    for b in range(B):
+        kept = np.asarray(keep[b]) != 0
+        kept[0] = True
+        t = x[b][kept]                                   # [L_b, D], ascending token order
+        qkv = layer_norm(t) @ Wqkv.T                     # [L_b, 3D]
+        q, k, v = qkv[:, :D], qkv[:, D:2 * D], qkv[:, 2 * D:]
+        att = np.zeros_like(t)
+        for h in range(H):
+            c = slice(h * d, (h + 1) * d)
+            s = scale * (q[:, c] @ k[:, c].T)
+            p = np.exp(s - s.max(axis=1, keepdims=True))
+            att[:, c] = (p / p.sum(axis=1, keepdims=True)) @ v[:, c]
+        hres = t + att @ Wo.T
+        z = layer_norm(hres) @ W1.T
+        y = hres + (0.5 * z * (1.0 + erf_v(z / sqrt(2.0)))) @ W2.T
+        out[b] = y[0]
+    return out

@@ -356,30 +356,136 @@ void oracle_mask_topk(const float *scores, int64_t B, int64_t L_full, const int3
     free(order);
 }
 
+/* Threshold-l2 on exact values.  Every f16, bf16 and f32 value is an integer
+ * multiple of 2^-149 (the smallest f32 subnormal), so every square, and every
+ * sum of squares, is an integer multiple of 2^-298.  The sum of squares of a
+ * token is therefore held exactly, as that integer, in a little-endian array
+ * of 32-bit limbs; with at most 2^24 elements below 2^128 in magnitude it is
+ * below 2^578, and 24 limbs (768 bits) hold it.  It is compared with tau^2,
+ * also exact, so no rounding and no order of summation enters the decision:
+ *     kept  <=>  j == 0  or  sqrt(sum of squares) >= tau.
+ * A NaN element makes the norm NaN, which is not >= tau (dropped); an
+ * infinite element without a NaN makes it infinite (kept). */
+#define L2_UNIT 298  /* the sums count units of 2^-298 */
+#define L2_LIMBS 24
+
+/* |v| = m * 2^e with m odd (v finite and nonzero). */
+static void odd_parts(double v, uint64_t *m, int *e)
+{
+    int k;
+    const double f = frexp(fabs(v), &k);        /* |v| = f * 2^k, 0.5 <= f < 1 */
+    uint64_t mm = (uint64_t)ldexp(f, 53);       /* exact: a double has 53 bits */
+    int ee = k - 53;
+    while ((mm & 1u) == 0) {
+        mm >>= 1;
+        ++ee;
+    }
+    *m = mm;
+    *e = ee;
+}
+
+/* Bits lo .. lo + 31 of v (zeros outside 0 .. 127; lo may be negative). */
+static uint32_t bits32(unsigned __int128 v, int lo)
+{
+    if (lo <= -32 || lo >= 128)
+        return 0;
+    if (lo < 0)
+        return (uint32_t)(v << (-lo));
+    return (uint32_t)(v >> lo);
+}
+
+/* acc += v * 2^shift (shift >= 0); the caller makes sure the sum fits. */
+static void big_add(uint32_t *acc, unsigned __int128 v, int shift)
+{
+    uint64_t carry = 0;
+    for (int i = 0; i < L2_LIMBS; ++i) {
+        const uint64_t sum = (uint64_t)acc[i] + bits32(v, 32 * i - shift) + carry;
+        acc[i] = (uint32_t)sum;
+        carry = sum >> 32;
+    }
+}
+
+static int bit_length(unsigned __int128 v)
+{
+    int n = 0;
+    while (v != 0) {
+        v >>= 1;
+        ++n;
+    }
+    return n;
+}
+
+/* a >= b for two L2_LIMBS-limb integers. */
+static int big_ge(const uint32_t *a, const uint32_t *b)
+{
+    for (int i = L2_LIMBS - 1; i >= 0; --i)
+        if (a[i] != b[i])
+            return a[i] > b[i];
+    return 1;
+}
+
+/* Is S * 2^-298 >= tau^2, for tau > 0 finite and S the sum in units? */
+static int sum_reaches(const uint32_t *S, double tau)
+{
+    uint64_t M;
+    int E;
+    odd_parts(tau, &M, &E);                      /* tau^2 = M^2 * 2^(2E) */
+    const unsigned __int128 M2 = (unsigned __int128)M * M;
+    const int shift = 2 * E + L2_UNIT;           /* tau^2 = M2 * 2^shift units */
+    uint32_t T[L2_LIMBS];
+    memset(T, 0, sizeof T);
+    if (shift >= 0) {
+        if (bit_length(M2) + shift > 32 * L2_LIMBS)
+            return 0;                            /* tau^2 >= 2^768 units, above any sum */
+        big_add(T, M2, shift);
+    } else {
+        /* S is a whole number of units: S >= M2 / 2^c  <=>  S >= ceil(M2 / 2^c) */
+        const int c = -shift;
+        unsigned __int128 q;
+        if (c >= 128)
+            q = 1;                               /* 0 < M2 / 2^c < 1 */
+        else
+            q = (M2 >> c) + ((M2 & ((((unsigned __int128)1) << c) - 1)) != 0);
+        big_add(T, q, 0);
+    }
+    return big_ge(S, T);
+}
+
 /* keep [B, L_full] <- Threshold-l2 of the tokens of x: token (b, j) is the C
- * elements starting at element (b * L_full + j) * tok_stride.  The sum of
- * squares is exact up to fp64 rounding (every square of an f16, bf16 or f32
- * element is exact in fp64).  Where it decides a keep bit, both sides must
- * round the same additions, so the sum is formed in the order the GPU kernel
- * uses: 32 partial sums over the elements c = l, l + 32, l + 64, ... in turn
- * (l = 0..31), then combined pairwise, partial l with partial l + 16, then
- * l + 8, l + 4, l + 2, l + 1.  The norm is the correctly rounded square root. */
+ * elements starting at element (b * L_full + j) * tok_stride. */
 void oracle_mask_l2(const void *x, int dtype, int64_t B, int64_t L_full, int64_t C, int64_t tok_stride,
                     double tau, uint8_t *keep)
 {
     for (int64_t t = 0; t < B * L_full; ++t) {
-        double part[32];
-        for (int l = 0; l < 32; ++l) {
-            part[l] = 0.0;
-            for (int64_t c = l; c < C; c += 32) {
-                const double v = load_elem(x, dtype, t * tok_stride + c);
-                part[l] = part[l] + v * v;
+        uint32_t S[L2_LIMBS];
+        memset(S, 0, sizeof S);
+        int has_nan = 0, has_inf = 0;
+        for (int64_t c = 0; c < C; ++c) {
+            const double v = load_elem(x, dtype, t * tok_stride + c);
+            if (isnan(v)) {
+                has_nan = 1;
+            } else if (isinf(v)) {
+                has_inf = 1;
+            } else if (v != 0.0) {
+                uint64_t m;
+                int e;
+                odd_parts(v, &m, &e);            /* e >= -149 for every f32 value */
+                if (2 * e + L2_UNIT < 0)
+                    abort();                     /* not an f16 / bf16 / f32 value */
+                big_add(S, (unsigned __int128)m * m, 2 * e + L2_UNIT);
             }
         }
-        for (int off = 16; off >= 1; off >>= 1)
-            for (int l = 0; l < off; ++l)
-                part[l] = part[l] + part[l + off];
-        const int64_t j = t % L_full;
-        keep[t] = (j == 0 || sqrt(part[0]) >= tau) ? 1 : 0;
+        int kept;
+        if (t % L_full == 0)
+            kept = 1;                            /* CLS */
+        else if (has_nan)
+            kept = 0;
+        else if (has_inf || !(tau > 0.0))
+            kept = 1;                            /* an infinite norm, or tau <= 0 */
+        else if (isinf(tau))
+            kept = 0;
+        else
+            kept = sum_reaches(S, tau);
+        keep[t] = (uint8_t)kept;
     }
 }

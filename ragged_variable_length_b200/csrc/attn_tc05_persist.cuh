@@ -322,7 +322,12 @@ __global__ void __launch_bounds__(kPersistThreads, 2)
             int n = 0;
             if (b < a.B) {
                 const int st = s_cu[b], len = s_cu[b + 1] - st;
-                if (st < 0 || len < 0 || len > a.max_seqlen) raise_status(RAGGED_DEV_BAD_SEQLENS);
+                // The tensor maps cover rows [0, B * max_seqlen): a sequence
+                // reaching past them (cu[0] != 0 can shift one there) would
+                // read zero fill, so it is flagged and skipped like the rest.
+                if (st < 0 || len < 0 || len > a.max_seqlen ||
+                    static_cast<int64_t>(st) + len > static_cast<int64_t>(a.B) * a.max_seqlen)
+                    raise_status(RAGGED_DEV_BAD_SEQLENS);
                 else n = ((len + kRows - 1) / kRows) * a.H;
             }
 #pragma unroll

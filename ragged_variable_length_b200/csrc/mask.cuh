@@ -37,15 +37,89 @@ __device__ __forceinline__ double widen<float>(const void* p, int64_t i) {
 constexpr int kMaskThreads = 256;   // 8 tokens per CTA, one warp each
 constexpr int kMaskMaxImages = 65535;   // images per launch (grid y)
 
+// ---- exact Threshold-l2 decision ------------------------------------------
+//
+// The keep bit is the exact comparison sum(x_c^2) >= tau^2 (tau > 0), so that
+// no summation order or rounding decides it.  A token's sum is first formed in
+// fp64 in whatever order the warp finds fast; every square of an f16, bf16 or
+// f32 value is exact in fp64 and only the additions round, so for n <= 2^24 +
+// 32 terms the sum is within a relative 2^-29 of the exact one.  Outside a
+// relative band of 2^-26 around tau^2 that settles the bit.  Inside it (ties
+// and near-ties only), one lane recomputes the sum exactly: every such value
+// is an integer multiple of 2^-149, so the sum of squares is an integer number
+// of units of 2^-298, below 2^578 units, held in 24 32-bit limbs, and tau^2 is
+// compared with it in the same units.
+constexpr int kL2Unit = 298;
+constexpr int kL2Limbs = 24;
+
+// |v| = m * 2^e with m odd; v a finite, nonzero, normal double.
+__device__ __forceinline__ void l2_odd_parts(double v, uint64_t& m, int& e) {
+    const uint64_t bits = static_cast<uint64_t>(__double_as_longlong(v)) & 0x7fffffffffffffffull;
+    m = (bits & 0xfffffffffffffull) | (1ull << 52);
+    e = static_cast<int>(bits >> 52) - 1075;
+    const int tz = __ffsll(static_cast<long long>(m)) - 1;
+    m >>= tz;
+    e += tz;
+}
+
+// acc += v * 2^shift, 0 <= shift, the result within kL2Limbs limbs.
+__device__ __noinline__ void l2_big_add(uint32_t* acc, unsigned __int128 v, int shift) {
+    const int w = shift >> 5, off = shift & 31;
+    uint32_t part[5];
+    const unsigned __int128 lo = v << off;                          // bits 0..127 of v * 2^off
+    const uint32_t top = off ? static_cast<uint32_t>(v >> (128 - off)) : 0u;   // bits 128..159
+#pragma unroll
+    for (int i = 0; i < 4; ++i) part[i] = static_cast<uint32_t>(lo >> (32 * i));
+    part[4] = top;
+    uint64_t carry = 0;
+    for (int i = w; i < kL2Limbs; ++i) {
+        const uint64_t sum = static_cast<uint64_t>(acc[i]) + (i - w < 5 ? part[i - w] : 0u) + carry;
+        acc[i] = static_cast<uint32_t>(sum);
+        carry = sum >> 32;
+    }
+}
+
+// Exact: does sum over c of x[base + c]^2 reach tau^2?  (0 < tau < 2^141, the
+// elements finite.)
+template <typename T>
+__device__ __noinline__ bool l2_exact_reaches(const void* x, int64_t base, int C, double tau) {
+    uint32_t S[kL2Limbs], Tq[kL2Limbs];
+    for (int i = 0; i < kL2Limbs; ++i) S[i] = Tq[i] = 0u;
+    for (int c = 0; c < C; ++c) {
+        const double v = widen<T>(x, base + c);
+        if (v == 0.0) continue;
+        uint64_t m;
+        int e;
+        l2_odd_parts(v, m, e);   // m < 2^24, e >= -149 for every f32 value
+        l2_big_add(S, static_cast<unsigned __int128>(m * m), 2 * e + kL2Unit);
+    }
+    uint64_t M;
+    int E;
+    l2_odd_parts(tau, M, E);
+    const unsigned __int128 M2 = static_cast<unsigned __int128>(M) * M;   // < 2^106
+    const int shift = 2 * E + kL2Unit;
+    if (shift >= 0) {
+        int bits = 0;
+        for (unsigned __int128 r = M2; r != 0; r >>= 1) ++bits;
+        if (bits + shift > 32 * kL2Limbs) return false;
+        l2_big_add(Tq, M2, shift);
+    } else {
+        const int c = -shift;   // S is whole units: S >= M2 / 2^c  <=>  S >= ceil(M2 / 2^c)
+        const unsigned __int128 q =
+            c >= 128 ? static_cast<unsigned __int128>(1)
+                     : (M2 >> c) + ((M2 & ((static_cast<unsigned __int128>(1) << c) - 1)) != 0);
+        l2_big_add(Tq, q, 0);
+    }
+    for (int i = kL2Limbs - 1; i >= 0; --i)
+        if (S[i] != Tq[i]) return S[i] > Tq[i];
+    return true;
+}
+
 // keep[b * L_full + j] for the tokens j of the images b = blockIdx.y (one warp
 // per token, blockIdx.x covering 8 tokens of the image); token (b, j) is the C
-// elements from element (b * L_full + j) * tok_stride.  The sum of squares is
-// formed in fp64 in a fixed order, so that the keep decision at the threshold
-// is reproducible: lane l adds the squares of elements l, l + 32, l + 64, ...
-// in turn (every square of an f16, bf16 or f32 element is exact in fp64), then
-// the 32 partial sums are combined pairwise with xor-shuffles 16, 8, 4, 2, 1.
-// Explicit round-to-nearest intrinsics keep the compiler from contracting the
-// multiply-add.
+// elements from element (b * L_full + j) * tok_stride.  Kept: CLS; a token
+// whose norm is infinite; otherwise, without a NaN element, sum x^2 >= tau^2
+// exactly (every token when tau <= 0).
 template <typename T>
 __global__ void __launch_bounds__(kMaskThreads)
     mask_l2_kernel(const void* __restrict__ x, int L_full, int C, int64_t tok_stride, double tau,
@@ -55,14 +129,34 @@ __global__ void __launch_bounds__(kMaskThreads)
     if (j >= L_full) return;   // warp-uniform
     const int64_t t = static_cast<int64_t>(blockIdx.y) * L_full + j;
     const int64_t base = t * tok_stride;
-    double ss = 0.0;
-    for (int c = lane; c < C; c += 32) {
-        const double v = widen<T>(x, base + c);
-        ss = __dadd_rn(ss, __dmul_rn(v, v));
+    double s0 = 0.0, s1 = 0.0;
+    int c = lane;
+    for (; c + 32 < C; c += 64) {
+        const double v0 = widen<T>(x, base + c), v1 = widen<T>(x, base + c + 32);
+        s0 = __dadd_rn(s0, __dmul_rn(v0, v0));
+        s1 = __dadd_rn(s1, __dmul_rn(v1, v1));
     }
+    if (c < C) {
+        const double v0 = widen<T>(x, base + c);
+        s0 = __dadd_rn(s0, __dmul_rn(v0, v0));
+    }
+    double ss = __dadd_rn(s0, s1);
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) ss = __dadd_rn(ss, __shfl_xor_sync(0xffffffffu, ss, off));
-    if (lane == 0) keep[t] = (j == 0 || __dsqrt_rn(ss) >= tau) ? 1 : 0;
+    // ss is the same in every lane: the decision below is warp-uniform.
+    bool kept;
+    if (j == 0) kept = true;
+    else if (isnan(ss)) kept = false;                    // a NaN element
+    else if (isinf(ss) || !(tau > 0.0)) kept = true;    // an infinite element (squares of finite values stay below 2^280)
+    else if (tau > 0x1p+140) kept = false;               // tau^2 > 2^280 > any finite sum
+    else if (tau < 0x1p-400) kept = ss > 0.0;            // tau^2 below the smallest nonzero square, 2^-298
+    else {
+        const double t2 = __dmul_rn(tau, tau);
+        if (ss > __dmul_rn(t2, 1.0 + 0x1p-26)) kept = true;
+        else if (ss < __dmul_rn(t2, 1.0 - 0x1p-26)) kept = false;
+        else kept = lane == 0 ? l2_exact_reaches<T>(x, base, C, tau) : false;
+    }
+    if (lane == 0) keep[t] = kept ? 1 : 0;
 }
 
 // The top-k order as one unsigned key per token, larger key = ranks earlier:

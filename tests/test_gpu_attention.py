@@ -203,6 +203,34 @@ def test_bad_cu_seqlens_are_flagged_and_skipped(kernel):
     assert rv.ragged_get_device_status() == 0     # reading clears the word
 
 
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+def test_persistent_flags_sequences_past_its_tensor_maps(dtype):
+    """cu_seqlens shifted by 100 rows (cu[0] != 0): the persistent kernel's TMA
+    maps cover rows [0, B * max_seqlen), so the last sequence, which ends past
+    them, is flagged and left untouched; the others are still correct."""
+    B, H, L = 4, 2, 197
+    rng = np.random.default_rng(88)
+    rows = 100 + B * L
+    qkv = synthetic.store(rng.standard_normal((rows, 3, H, 64)).astype(np.float32), dtype)
+    dev = to_device(qkv, dtype)
+    cu_h = np.array([100 + i * L for i in range(B + 1)], dtype=np.int32)
+    cu = torch.from_numpy(cu_h).cuda()
+    out = torch.full((rows, H, 64), float("nan"), dtype=TORCH_DTYPE[dtype], device="cuda")
+    rv.ragged_get_device_status()
+    prev = rv.ragged_set_attn_kernel(rv.RAGGED_ATTN_PERSISTENT)
+    try:
+        rv.ragged_attn_fwd(dev[:, 0], dev[:, 1], dev[:, 2], cu, L, 0.125, out=out)
+    finally:
+        rv.ragged_set_attn_kernel(prev)
+    torch.cuda.synchronize()
+    assert rv.ragged_get_device_status() & rv.RAGGED_DEV_BAD_SEQLENS
+    assert torch.isnan(out[:100]).all() and torch.isnan(out[int(cu_h[3]):]).all()
+    ref = oracle.attention(qkv[:, 0], qkv[:, 1], qkv[:, 2], cu_h, dtype, 0.125, seqs=[0, 1, 2])
+    got = to_f64(out[100:int(cu_h[3])])
+    err, bound = attn_error(got, ref[100:int(cu_h[3])], dtype)
+    assert err <= bound, f"{err:.3e} > {bound:.3e}"
+
+
 def test_pipeline_call_and_graph_replay_match_separate_calls():
     w = synthetic.serving(4, 0.25)
     cu_ref, out_ref, cls_ref, _ = run_pipeline(w)

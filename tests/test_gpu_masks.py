@@ -42,6 +42,43 @@ def test_mask_l2_at_the_threshold():
     assert rv.ragged_mask_l2(torch.from_numpy(x).cuda(), 5.0).cpu().tolist() == [[1, 1, 1, 0, 1]]
 
 
+@pytest.mark.parametrize("dtype", ["f16", "bf16", "f32"])
+def test_mask_l2_exact_at_and_next_to_each_norm(dtype):
+    """Each token's own norm as tau (the double nearest it, and one ulp either
+    side), so every decision falls in the band where the kernel's fp64 sum
+    cannot decide and its exact integer sum must: bit-exact against the oracle."""
+    rng = synthetic.rng_for(3007, ["f16", "bf16", "f32"].index(dtype))
+    B, L, C = 2, 12, 384
+    x = synthetic.store(rng.standard_normal((B, L, C)).astype(np.float32), dtype)
+    xf = oracle.decode(x, dtype).reshape(B, L, C)
+    xd = to_device(x, dtype)
+    norms = np.sqrt((xf * xf).sum(2))
+    for b in range(B):
+        for j in (1, 5, 11):
+            t0 = float(norms[b, j])
+            for tau in (float(np.nextafter(t0, 0.0)), t0, float(np.nextafter(t0, np.inf))):
+                got = rv.ragged_mask_l2(xd, tau).cpu().numpy()
+                assert np.array_equal(got, oracle.mask_l2(x, dtype, tau)), (b, j, tau)
+
+
+def test_mask_l2_where_fp64_sums_round_subnormals_nan_inf():
+    x = np.zeros((1, 8, 64), dtype=np.float32)
+    x[0, 1, :4] = [1.0, 2.0 ** -26, 2.0 ** -26, 2.0 ** -52]     # sum of squares (1 + 2^-52)^2 exactly
+    x[0, 2, 0] = 1.0
+    x[0, 2, 1:17] = 2.0 ** -30                                   # 1 + 2^-56
+    x[0, 3, 3] = 2.0 ** -149                                     # square 2^-298
+    x[0, 4, 0], x[0, 4, 63] = 2.0 ** -149, 2.0 ** -149
+    x[0, 5, 0], x[0, 5, 1] = np.nan, 100.0
+    x[0, 6, 2] = -np.inf
+    x[0, 7, :] = 0.625                                           # norm 5 exactly
+    xd = torch.from_numpy(x).cuda()
+    for tau in (1.0 + 2.0 ** -52, float(np.nextafter(1.0 + 2.0 ** -52, 2.0)), 1.0, float(np.nextafter(1.0, 2.0)),
+                2.0 ** -149, float(np.nextafter(2.0 ** -149, 1.0)), 2.0 ** -149 * 2 ** 0.5, 5.0, 1e-300, 1e300,
+                float("inf"), 0.0, -1.0):
+        got = rv.ragged_mask_l2(xd, tau).cpu().numpy()
+        assert np.array_equal(got, oracle.mask_l2(x, "f32", tau)), tau
+
+
 def test_mask_l2_on_a_strided_view():
     """Norm of the q part of a dense fused [B, L, 3, H, 64] buffer (token stride 3 * H * 64)."""
     w = synthetic.serving(4, 0.0)

@@ -10,6 +10,7 @@ serves, radpulse "Integrated pack pipeline", without spelling out a rule):
 Each pin ties the oracle to something other than itself: a sort by numpy's
 lexsort, exact rational arithmetic, closed cases and invariants.
 """
+import math
 from fractions import Fraction
 
 import numpy as np
@@ -115,6 +116,60 @@ def test_l2_matches_exact_arithmetic(dtype):
         for j in range(L):
             want = 1 if j == 0 or _exact_norm_sq(xf[b, j]) >= tau_sq else 0
             assert keep[b, j] == want, (b, j)
+
+
+@pytest.mark.parametrize("dtype", ["f16", "bf16", "f32"])
+def test_l2_exact_at_and_next_to_tau(dtype):
+    """Thresholds at, one ulp below and one ulp above the double nearest each
+    token's norm: the decision must be the exact rational comparison
+    sum(x^2) >= tau^2 (Python fractions), whatever fp64 rounding would say."""
+    rng = synthetic.rng_for(2004, ["f16", "bf16", "f32"].index(dtype))
+    B, L, C = 2, 9, 384
+    x = synthetic.store(rng.standard_normal((B, L, C)).astype(np.float32), dtype)
+    xf = oracle.decode(x, dtype).reshape(B, L, C)
+    for b in range(B):
+        for j in range(1, L):
+            exact = _exact_norm_sq(xf[b, j])
+            t0 = math.sqrt(float(exact))
+            for tau in (np.nextafter(t0, 0.0), t0, np.nextafter(t0, np.inf)):
+                keep = oracle.mask_l2(x, dtype, float(tau))
+                want = 1 if exact >= Fraction(float(tau)) ** 2 else 0
+                assert keep[b, j] == want, (b, j, tau)
+
+
+def test_l2_decides_where_fp64_sums_round():
+    """Sums of squares that fp64 addition rounds: 1 + 2^-51 + 2^-104 (squares
+    of 1, 2^-26, 2^-26, 2^-52) is exactly (1 + 2^-52)^2; sixteen squares of
+    2^-30 added to 1 vanish in any fp64 order that starts from 1."""
+    x = np.zeros((1, 3, 64), dtype=np.float32)
+    x[0, 1, :4] = [1.0, 2.0 ** -26, 2.0 ** -26, 2.0 ** -52]
+    x[0, 2, 0] = 1.0
+    x[0, 2, 1:17] = 2.0 ** -30
+    tau = 1.0 + 2.0 ** -52
+    assert Fraction(tau) ** 2 == _exact_norm_sq(x[0, 1])
+    assert oracle.mask_l2(x, "f32", tau).tolist() == [[1, 1, 0]]
+    assert oracle.mask_l2(x, "f32", float(np.nextafter(tau, 2.0))).tolist() == [[1, 0, 0]]
+    # row 2: 1 + 16 * 2^-60 = 1 + 2^-56 > 1, so it reaches tau = 1 and not the next double
+    assert oracle.mask_l2(x, "f32", 1.0).tolist() == [[1, 1, 1]]
+    assert oracle.mask_l2(x, "f32", float(np.nextafter(1.0, 2.0))).tolist() == [[1, 1, 0]]
+
+
+def test_l2_subnormals_nan_and_infinity():
+    tiny = np.float32(2.0 ** -149)                 # the smallest f32 subnormal; its square is 2^-298
+    x = np.zeros((1, 5, 8), dtype=np.float32)
+    x[0, 1, 3] = tiny
+    x[0, 2, 0], x[0, 2, 5] = tiny, tiny            # norm 2^-149 * sqrt(2)
+    x[0, 3, 0], x[0, 3, 1] = np.nan, 100.0
+    x[0, 4, 2] = -np.inf
+    t = 2.0 ** -149
+    assert oracle.mask_l2(x, "f32", t).tolist() == [[1, 1, 1, 0, 1]]
+    assert oracle.mask_l2(x, "f32", float(np.nextafter(t, 1.0))).tolist() == [[1, 0, 1, 0, 1]]
+    assert oracle.mask_l2(x, "f32", t * math.sqrt(2.0) * (1 + 2.0 ** -40)).tolist() == [[1, 0, 0, 0, 1]]
+    # a threshold far below the smallest nonzero square, and one far above any sum
+    assert oracle.mask_l2(x, "f32", 1e-300).tolist() == [[1, 1, 1, 0, 1]]
+    assert oracle.mask_l2(x, "f32", 1e300).tolist() == [[1, 0, 0, 0, 1]]
+    # an infinite norm reaches even an infinite tau (inf >= inf); a NaN norm reaches nothing
+    assert oracle.mask_l2(x, "f32", float("inf")).tolist() == [[1, 0, 0, 0, 1]]
 
 
 def test_l2_boundary_and_closed_cases():

@@ -37,9 +37,15 @@ MUTANTS = {
     "topk_nan_ranks_first": ("return nb; /* every number ranks before NaN */", "return na; /* every number ranks before NaN */"),
     "topk_ascending": ("        return a > b;", "        return a < b;"),
     "topk_one_too_few": ("for (int64_t r = 0; r < k - 1; ++r)", "for (int64_t r = 0; r < k - 2; ++r)"),
-    "l2_strict_threshold": ("sqrt(part[0]) >= tau", "sqrt(part[0]) > tau"),
-    "l2_last_element_dropped": ("for (int64_t c = l; c < C; c += 32)", "for (int64_t c = l; c < C - 1; c += 32)"),
-    "l2_cls_not_forced": ("keep[t] = (j == 0 || sqrt(part[0]) >= tau) ? 1 : 0;", "keep[t] = (sqrt(part[0]) >= tau) ? 1 : 0;"),
+    "l2_strict_threshold": ("            return a[i] > b[i];\n    return 1;", "            return a[i] > b[i];\n    return 0;"),
+    "l2_last_element_dropped": ("for (int64_t c = 0; c < C; ++c) {\n            const double v = load_elem(x, dtype, t * tok_stride + c);",
+                                "for (int64_t c = 0; c < C - 1; ++c) {\n            const double v = load_elem(x, dtype, t * tok_stride + c);"),
+    "l2_cls_not_forced": ("if (t % L_full == 0)\n            kept = 1;", "if (t % L_full == -1)\n            kept = 1;"),
+    "l2_square_doubled": ("big_add(S, (unsigned __int128)m * m, 2 * e + L2_UNIT);",
+                          "big_add(S, (unsigned __int128)m * m, 2 * e + L2_UNIT + 1);"),
+    "l2_carry_lost": ("        carry = sum >> 32;", "        carry = 0;"),
+    "l2_tau_rounded_down": ("q = (M2 >> c) + ((M2 & ((((unsigned __int128)1) << c) - 1)) != 0);", "q = (M2 >> c);"),
+    "l2_nan_kept": ("        else if (has_nan)\n            kept = 0;", "        else if (has_nan)\n            kept = 1;"),
 }
 
 
@@ -54,12 +60,14 @@ def _pin_calls():
     for keep in pins._random_masks():
         calls.append(lambda keep=keep: pins.test_seqlens_matches_flatnonzero(keep))
         calls.append(lambda keep=keep: pins.test_pack_unpack_roundtrip(keep))
-    calls += [mpins.test_topk_closed_cases, mpins.test_topk_counts_and_cls, mpins.test_l2_boundary_and_closed_cases]
+    calls += [mpins.test_topk_closed_cases, mpins.test_topk_counts_and_cls, mpins.test_l2_boundary_and_closed_cases,
+              mpins.test_l2_decides_where_fp64_sums_round, mpins.test_l2_subnormals_nan_and_infinity]
     for ties in (False, True):
         for nans in (False, True):
             calls.append(lambda ties=ties, nans=nans: mpins.test_topk_matches_lexsort(ties, nans))
     for dt in ("f16", "bf16", "f32"):
         calls.append(lambda dt=dt: mpins.test_l2_matches_exact_arithmetic(dt))
+        calls.append(lambda dt=dt: mpins.test_l2_exact_at_and_next_to_tau(dt))
     return calls
 
 
