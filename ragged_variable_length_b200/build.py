@@ -18,6 +18,8 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libragged.so")
+# The same sources with RAGGED_TEST_HOOKS: failure-path switches for the tests.
+HOOKS_LIB = os.path.join(HERE, "libragged_testhooks.so")
 MAIN = os.path.join(CSRC, "ragged_api.cu")
 
 ARCH_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -35,17 +37,19 @@ def sources() -> list:
                   glob.glob(os.path.join(INCLUDE, "*.h")))
 
 
-def stale() -> bool:
-    if not os.path.exists(LIB):
+def stale(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return any(os.path.getmtime(s) > t for s in sources())
 
 
-def command(out: str, ptxas_verbose: bool = False) -> list:
+def command(out: str, ptxas_verbose: bool = False, test_hooks: bool = False) -> list:
     cmd = [nvcc(), *ARCH_FLAGS, "-O3", "-lineinfo", "-std=c++17", "-shared", "-Xcompiler", "-fPIC",
            "-Xcompiler", "-fvisibility=hidden", "--expt-relaxed-constexpr", "-cudart", "static",
            f"-I{INCLUDE}", f"-I{CSRC}", "-DRAGGED_BUILD", MAIN, "-o", out]
+    if test_hooks:
+        cmd.insert(-3, "-DRAGGED_TEST_HOOKS")
     if ptxas_verbose:
         cmd[1:1] = ["-Xptxas", "-v"]
     return cmd
@@ -72,21 +76,32 @@ def build_fastcall(force: bool = False) -> str:
     return out
 
 
-def build(force: bool = False, ptxas_verbose: bool = False) -> str:
-    build_fastcall(force)
-    if not force and not stale():
-        return LIB
-    tmp = f"{LIB}.{os.getpid()}.tmp"
-    proc = subprocess.run(command(tmp, ptxas_verbose), capture_output=True, text=True)
+def _compile(lib: str, force: bool, ptxas_verbose: bool, test_hooks: bool) -> str:
+    if not force and not stale(lib):
+        return lib
+    tmp = f"{lib}.{os.getpid()}.tmp"
+    proc = subprocess.run(command(tmp, ptxas_verbose, test_hooks), capture_output=True, text=True)
     if proc.returncode != 0:
         sys.stderr.write(proc.stdout + proc.stderr)
-        raise RuntimeError("nvcc failed building libragged.so")
+        raise RuntimeError(f"nvcc failed building {os.path.basename(lib)}")
     if ptxas_verbose:
         sys.stderr.write(proc.stdout + proc.stderr)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
+
+
+def build(force: bool = False, ptxas_verbose: bool = False) -> str:
+    build_fastcall(force)
+    return _compile(LIB, force, ptxas_verbose, False)
+
+
+def build_test_hooks(force: bool = False) -> str:
+    """libragged_testhooks.so: the library with the failure-path test switches."""
+    return _compile(HOOKS_LIB, force, False, True)
 
 
 if __name__ == "__main__":
     build(force="--force" in sys.argv, ptxas_verbose="--verbose-ptxas" in sys.argv)
     print(LIB)
+    if "--test-hooks" in sys.argv:
+        print(build_test_hooks(force="--force" in sys.argv))

@@ -27,6 +27,22 @@ constexpr int kQBytes = kRows * 128;               // 16 KB
 constexpr int kKVTileBytes = kTileN * 128;         // 8 KB
 constexpr uint32_t kSpinLimit = 1u << 22;
 
+#ifdef RAGGED_TEST_HOOKS
+// Test builds only (libragged_testhooks.so, never the product library): a
+// test can shorten every bounded wait and tell a kernel's producer to issue
+// nothing, so that the waits on it expire without any fault, and then check
+// that the status word reports it, TMEM comes back and the next launch is
+// exact.  g_test_hook: 1 = the persistent kernel's load warp issues no load;
+// 2 = the per-tile kernel's MMA thread issues no product.
+__device__ uint32_t g_test_spin_limit = kSpinLimit;
+__device__ int g_test_hook = 0;
+__device__ __forceinline__ uint32_t spin_limit() { return g_test_spin_limit; }
+__device__ __forceinline__ bool test_hook(int which) { return g_test_hook == which; }
+#else
+__device__ __forceinline__ constexpr uint32_t spin_limit() { return kSpinLimit; }
+__device__ __forceinline__ constexpr bool test_hook(int) { return false; }
+#endif
+
 // ---- instruction and shared-memory descriptors -------------------------------
 
 // kind::f16 instruction descriptor: fp32 accumulate, A/B format (0 = f16,
@@ -80,7 +96,8 @@ __device__ __forceinline__ void mbar_init(uint32_t mbar, uint32_t count) {
 // Waits for the phase with the given parity to complete; false after the
 // bounded number of polls.
 __device__ __forceinline__ bool mbar_wait(uint32_t mbar, uint32_t parity) {
-    for (uint32_t i = 0; i < kSpinLimit; ++i) {
+    const uint32_t limit = spin_limit();
+    for (uint32_t i = 0; i < limit; ++i) {
         uint32_t done;
         asm volatile(
             "{\n\t.reg .pred p;\n\t"
@@ -314,7 +331,7 @@ __global__ void __launch_bounds__(kStreamThreads, 2)
 
     if (mma_warp) {
         // ---------------- MMA issuer (one thread) ----------------
-        if ((tid & 31) == 0) {
+        if ((tid & 31) == 0 && !test_hook(2)) {
             const uint32_t idesc_qk = make_idesc(Cvt<T>::kFormat, 0, kTileN);
             const uint32_t idesc_pv = make_idesc(Cvt<T>::kFormat, 1, 64);
             auto issue_pv = [&](int t) {   // P V of tile t, once P(t) is ready

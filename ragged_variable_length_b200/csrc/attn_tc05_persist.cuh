@@ -359,7 +359,7 @@ __global__ void __launch_bounds__(kPersistThreads, 2)
         auto publish_copies = [&](uint32_t mbar) { cp_async_arrive_noinc(mbar); };
         uint32_t g = 0;
         int k = 0;
-        bool ok = true;
+        bool ok = !test_hook(1);
         for (int j = blockIdx.x; ok && j < total; j += gridDim.x, ++k) {
             if (__any_sync(kFullMask, *fail_flag != 0)) break;
             const Item it = decode_item(j, s_cu, s_ip, a.B, a.H);

@@ -691,4 +691,15 @@ ragged_status ragged_pipeline_noalloc(const void* dense_qkv, const uint8_t* keep
 }
 
 
+#ifdef RAGGED_TEST_HOOKS
+// Test builds only; declared in ragged_test_hooks.h.
+RAGGED_API ragged_status ragged_test_set_hooks(int32_t hook, uint32_t spin_limit) {
+    if (hook < 0 || hook > 2 || spin_limit == 0) return fail(RAGGED_ERR_INVALID_ARG, "bad test hook settings");
+    ragged_status st = cuda_check(cudaMemcpyToSymbol(ragged::tc05::g_test_hook, &hook, sizeof hook), "test hook");
+    if (st != RAGGED_OK) return st;
+    return cuda_check(cudaMemcpyToSymbol(ragged::tc05::g_test_spin_limit, &spin_limit, sizeof spin_limit),
+                      "test spin limit");
+}
+#endif
+
 }  // extern "C"

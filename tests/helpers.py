@@ -63,3 +63,27 @@ def attn_error(gpu: np.ndarray, ref: np.ndarray, dtype: str):
     bound = bound_16bit(ref, dtype)
     i = int(np.argmax(diff / bound))
     return float(diff.flat[i]), float(bound.flat[i])
+
+
+def round_to_format(x: np.ndarray, dtype: str) -> np.ndarray:
+    """x (float64) rounded to nearest even in f16 or bf16, returned as float64.
+    Normal range only (the attention outputs here), straight from float64 so
+    that no intermediate rounding enters."""
+    bits = 7 if dtype == "bf16" else 10
+    m, e = np.frexp(x)                                # x = m * 2^e, 0.5 <= |m| < 1
+    return np.ldexp(np.round(np.ldexp(m, bits + 1)), e - bits - 1)   # np.round: half to even
+
+
+def ulps_from_rounded(gpu: np.ndarray, ref: np.ndarray, dtype: str, floor: float = 2.0 ** -10) -> int:
+    """Largest distance, in units in the last place of the 16-bit format,
+    between each GPU output and the oracle value correctly rounded to that
+    format.  Elements with |oracle| below `floor` are left out: near zero a
+    unit in the last place shrinks without limit, while the absolute bound of
+    attn_error already covers them."""
+    sel = np.abs(ref) >= floor
+    if not sel.any():
+        return 0
+    r = round_to_format(ref[sel], dtype)
+    bits = 7 if dtype == "bf16" else 10
+    ulp = np.ldexp(1.0, np.frexp(np.abs(r))[1] - bits - 1)
+    return int(np.max(np.round(np.abs(gpu[sel] - r) / ulp)))

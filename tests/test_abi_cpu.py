@@ -211,3 +211,14 @@ def test_binding_fails_loudly_without_the_library():
     assert not os.path.exists(missing)
     with pytest.raises(RuntimeError, match="missing"):
         rv.load(missing)
+
+
+def test_test_hooks_live_only_in_the_test_build():
+    """The failure-path switches are compiled into libragged_testhooks.so only."""
+    hooks = rbuild.build_test_hooks()
+    prod = os.popen(f"nm -D --defined-only {rv.LIB_PATH}").read()
+    test = os.popen(f"nm -D --defined-only {hooks}").read()
+    assert "ragged_test_set_hooks" not in prod
+    assert re.search(r" T ragged_test_set_hooks\b", test)
+    header = open(os.path.join(ROOT, "include", "ragged_test_hooks.h")).read()
+    assert "RAGGED_API ragged_status ragged_test_set_hooks(" in header
