@@ -336,6 +336,51 @@ def run_ours(args, rank, world, dist):
         entry["roofline_frac"] = round(t_roof_case / dev_s, 4)
         detail[f"b{B}_p{int(p * 100)}"] = entry
 
+    # ---- where the host side of a headline call goes ----
+    # A headline call is graph launch + kernel + stream synchronisation.  The
+    # same pattern around a graph holding one trivial kernel (a one-element
+    # fill) gives its floor; enqueue-only and idle-synchronise times split it.
+    def host_split(n=2000):
+        tiny = torch.zeros(1, device=dev)
+        side = torch.cuda.Stream()
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            tiny.fill_(1.0)
+            g_empty = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g_empty, stream=side):
+                tiny.fill_(1.0)
+        stream.wait_stream(side)
+        torch.cuda.synchronize()
+        pl = pipes[0][len(CASES) - 1]
+        enq, idle, empty_call, call = [], [], [], []
+        for r in range(n):
+            torch.cuda.synchronize()
+            t0 = time.perf_counter()
+            pl.replay()
+            t1 = time.perf_counter()
+            stream.synchronize()
+            enq.append((t1 - t0) * 1e6)
+            t0 = time.perf_counter()
+            stream.synchronize()
+            idle.append((time.perf_counter() - t0) * 1e6)
+            t0 = time.perf_counter()
+            g_empty.replay()
+            stream.synchronize()
+            empty_call.append((time.perf_counter() - t0) * 1e6)
+            t0 = time.perf_counter()
+            pl.replay()
+            stream.synchronize()
+            call.append((time.perf_counter() - t0) * 1e6)
+        med = lambda xs: round(statistics.median(xs), 2)
+        return {"case": f"b{CASES[-1][0]}_p{int(CASES[-1][1] * 100)}", "calls": n,
+                "graph_replay_enqueue_us": med(enq), "stream_sync_idle_us": med(idle),
+                "empty_kernel_graph_call_us": med(empty_call), "fused_graph_call_us": med(call),
+                "note": "median over calls; empty_kernel_graph_call_us is the floor of graph launch + "
+                        "one-kernel execution + synchronisation on this host, the rest of a call is the "
+                        "fused kernel beyond a trivial one"}
+
+    hsplit = optional(host_split)
+
     # ---- end to end from pinned host buffers ----
     host_in = {}
     for c in range(ncopies):
@@ -485,8 +530,31 @@ def run_ours(args, rank, world, dist):
             torch.cuda.empty_cache()
         return larger
 
+    # ---- per-launch floor of the attention kernels: one sequence of one token ----
+    def launch_floor():
+        w = synthetic.make_workload("one_token", 1, 1, 12, [1], "bf16", 1002, 9)
+        pl = rv.Pipeline(1, 1, 12, torch.bfloat16, device=dev, flags=rv.RAGGED_PIPELINE_SPLIT)
+        pl.dense_qkv.view(torch.int16).copy_(torch.from_numpy(w.qkv.view(np.int16)).to(dev))
+        pl.keep.copy_(torch.from_numpy(w.keep).to(dev))
+        pl()
+        torch.cuda.synchronize()
+        tiny = torch.zeros(1, device=dev)
+        res = {"empty_torch_kernel_us": round(graph_time([lambda strm: tiny.fill_(1.0)] * 32, replays=10) * 1e6, 2)}
+        for kname, kcode in (("streaming", rv.RAGGED_ATTN_STREAMING), ("resident", rv.RAGGED_ATTN_RESIDENT),
+                             ("tcgen05", rv.RAGGED_ATTN_TCGEN05), ("persistent", rv.RAGGED_ATTN_PERSISTENT)):
+            prev = rv.ragged_set_attn_kernel(kcode)
+            try:
+                res[kname + "_us"] = round(graph_time([attn_launcher(pl, w)] * 32, replays=10) * 1e6, 2)
+            finally:
+                rv.ragged_set_attn_kernel(prev)
+        res["note"] = ("average per launch of 32 back-to-back launches in a CUDA graph: attention on one "
+                       "1-token sequence with 12 heads (bf16), the fixed cost a launch pays whatever its work")
+        return res
+
     single = world == 1 and not args.quick
     larger = optional(measure_larger) if single else {}
+    if single and isinstance(larger, dict) and "error" not in larger:
+        larger["launch_floor"] = optional(launch_floor)
 
     # ---- padded PyTorch SDPA baseline, same calls, same synchronisation ----
     padded = optional(lambda: padded_baseline(args, pipes, workloads, ncopies, stream))
@@ -519,6 +587,7 @@ def run_ours(args, rank, world, dist):
           "direct_call_us_per_call": round(direct_us, 3),
           "warm_us_per_call": round(warm_us, 3),
           "per_case": detail,
+          "host_split": hsplit,
           "padded_sdpa": padded,
           "comparators": comps,
           "mask_producers": masks,

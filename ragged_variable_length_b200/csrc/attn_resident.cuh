@@ -123,14 +123,16 @@ struct DenseRows {
             const int j = threadIdx.x + i * kThreads;
             mine[i] = j < L_full ? kb[j] : 0;
         }
-        // Pull this head's q/k/v rows of the image towards L2 while the mask is
-        // ranked; the CTAs of one (image, head) share the prefetches.
+        // Pull this head's q/k/v rows of the surviving tokens towards L2 while
+        // the mask is ranked; the CTAs of one (image, head) share the
+        // prefetches.  Each prefetch waits only for its own token's keep byte,
+        // so dropped tokens' rows are never read.
         const int share = gridDim.x;
         const int64_t row_elems = 3LL * H * kHeadDim;
         for (int j = blockIdx.x + share * (threadIdx.x / 3); j < L_full; j += share * (kThreads / 3)) {
             if (threadIdx.x >= (kThreads / 3) * 3) break;
             const uint16_t* p = dense + (row0 + j) * row_elems + ((threadIdx.x % 3) * H + h) * kHeadDim;
-            asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+            if (j == 0 || kb[j] != 0) asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
         }
         int forced = 0;
         for (int i = threadIdx.x; i < b; i += kThreads) forced += keep[static_cast<int64_t>(i) * L_full] == 0;
