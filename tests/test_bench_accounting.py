@@ -100,7 +100,12 @@ def test_recorded_traffic_is_withheld_when_sources_change(monkeypatch):
     """The committed record is reported while the fused kernel's sources hash
     to the recorded value, and withheld (None) once they do not, or when the
     record is missing."""
-    assert bench.recorded_traffic() == 1100992
+    recorded = None
+    with open(bench.TRAFFIC_RECORD) as f:
+        for line in f:
+            if line.startswith("dram_bytes_per_launch_mean:"):
+                recorded = int(line.split(":", 1)[1])
+    assert recorded is not None and bench.recorded_traffic() == recorded
     monkeypatch.setattr(bench, "fused_source_hash", lambda: "0" * 64)
     assert bench.recorded_traffic() is None
     monkeypatch.undo()
