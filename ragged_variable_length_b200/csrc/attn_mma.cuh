@@ -58,7 +58,10 @@ __global__ void __launch_bounds__(kThreads)
                     uint16_t* __restrict__ out, int64_t out_tok_stride,
                     uint16_t* __restrict__ cls_out) {
     extern __shared__ __align__(128) uint8_t smem[];
-    const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    // The query tile is the slowest grid index: a launch is sized by the host
+    // bound max_seqlen, and with short sequences most CTAs of the later query
+    // tiles exit at once, so the ones with work are all dispatched first.
+    const int qt = blockIdx.z, h = blockIdx.x, b = blockIdx.y;
     int start, len;
     if (!read_sequence(cu, b, max_seqlen, start, len)) return;
     const int q0 = qt * kBlockM;
