@@ -566,8 +566,8 @@ ragged_status ragged_attn_fwd(const void* q, const void* k, const void* v, int64
                                               1, s);
     }
     using namespace ragged::mma_attn;
-    const dim3 grid(static_cast<unsigned>((max_seqlen + kBlockM - 1) / kBlockM), static_cast<unsigned>(H),
-                    static_cast<unsigned>(B));
+    const dim3 grid(static_cast<unsigned>(H), static_cast<unsigned>(B),
+                    static_cast<unsigned>((max_seqlen + kBlockM - 1) / kBlockM));
     const float scale_log2 = scale * 1.4426950408889634f;
     if (dtype == RAGGED_F16) {
         st = ensure_smem(attn_fwd_kernel<__half>, kSmemBytes, g_mma_f16_smem);
