@@ -212,7 +212,10 @@ def run_ours(args, rank, world, dist):
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
     torch.cuda.set_device(dev)
     rv.load()  # fails loudly if the CUDA library is missing
-    stream = torch.cuda.current_stream()
+    # A created stream (the library records its pipeline graphs on one; the
+    # legacy default stream cannot be captured) is current for everything below.
+    stream = torch.cuda.Stream(device=dev)
+    torch.cuda.set_stream(stream)
     hbm_peak, bf16_peak, peak_kind = peaks()
 
     # ---- inputs: enough copies of the 12 serving batches to exceed 2x L2 ----
@@ -229,14 +232,21 @@ def run_ours(args, rank, world, dist):
             pipes[c].append(pl)
     torch.cuda.synchronize()
 
-    # Every pipeline is also recorded as a CUDA graph (one kernel node); a
-    # call is then one graph launch plus a wait for completion.
+    # Every pipeline is also recorded as a CUDA graph (one kernel node), twice:
+    # by torch (Pipeline.capture) and by libragged (Pipeline.record).  A
+    # headline call is one crossing into libragged that launches its graph and
+    # waits for it (ragged_pipeline_graph_launch with RAGGED_PIPELINE_SYNC).
     for c in range(ncopies):
         for pl in pipes[c]:
             pl.capture()
+            pl.record()
     torch.cuda.synchronize()
 
     def step(s):
+        for pl in pipes[s % ncopies]:
+            pl.launch(sync=True)
+
+    def step_torch_graph(s):
         for pl in pipes[s % ncopies]:
             pl.replay()
             stream.synchronize()
@@ -248,6 +258,7 @@ def run_ours(args, rank, world, dist):
     for s in range(args.warmup):
         step(s)
         step_direct(s)
+        step_torch_graph(s)
     try:
         sampler = ClockSampler("GPU-" + str(torch.cuda.get_device_properties(dev).uuid))
     except Exception:
@@ -284,6 +295,19 @@ def run_ours(args, rank, world, dist):
     direct_ms = max_over_ranks(d0.elapsed_time(d1), dist, dev)
     direct_us = us_per_call(direct_ms, args.steps, len(CASES), world)
 
+    # The same calls through torch's graph of the pipeline: replay, then a
+    # stream synchronisation (two crossings into torch per call).
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    g0.record(stream)
+    for s in range(args.steps):
+        step_torch_graph(s)
+    g1.record(stream)
+    torch.cuda.synchronize()
+    torch_graph_us = us_per_call(max_over_ranks(g0.elapsed_time(g1), dist, dev), args.steps, len(CASES), world)
+
     # Warm, reported separately: the same graph calls on one input copy only,
     # whose 12 batches (about 12 MiB) stay in L2 from one step to the next.
     for _ in range(args.warmup):
@@ -319,7 +343,7 @@ def run_ours(args, rank, world, dist):
             host.append((h1 - h0) * 1e6)
             dev_t.append(a.elapsed_time(b) * 1e3)
             t0 = time.perf_counter()
-            pl.run_sync()
+            pl.launch(sync=True)
             tot.append((time.perf_counter() - t0) * 1e6)
         entry = {"calls": reps}
         for name, xs in (("host", host), ("device", dev_t), ("total", tot)):
@@ -352,7 +376,7 @@ def run_ours(args, rank, world, dist):
         stream.wait_stream(side)
         torch.cuda.synchronize()
         pl = pipes[0][len(CASES) - 1]
-        enq, idle, empty_call, call = [], [], [], []
+        enq, idle, empty_call, call, lib_call = [], [], [], [], []
         for r in range(n):
             torch.cuda.synchronize()
             t0 = time.perf_counter()
@@ -371,13 +395,19 @@ def run_ours(args, rank, world, dist):
             pl.replay()
             stream.synchronize()
             call.append((time.perf_counter() - t0) * 1e6)
+            t0 = time.perf_counter()
+            pl.launch(sync=True)
+            lib_call.append((time.perf_counter() - t0) * 1e6)
         med = lambda xs: round(statistics.median(xs), 2)
         return {"case": f"b{CASES[-1][0]}_p{int(CASES[-1][1] * 100)}", "calls": n,
                 "graph_replay_enqueue_us": med(enq), "stream_sync_idle_us": med(idle),
                 "empty_kernel_graph_call_us": med(empty_call), "fused_graph_call_us": med(call),
+                "fused_library_graph_call_us": med(lib_call),
                 "note": "median over calls; empty_kernel_graph_call_us is the floor of graph launch + "
-                        "one-kernel execution + synchronisation on this host, the rest of a call is the "
-                        "fused kernel beyond a trivial one"}
+                        "one-kernel execution + synchronisation on this host through torch, the rest of a "
+                        "call is the fused kernel beyond a trivial one; fused_graph_call_us goes through "
+                        "torch (replay + synchronize), fused_library_graph_call_us is the headline call "
+                        "(one crossing: ragged_pipeline_graph_launch with RAGGED_PIPELINE_SYNC)"}
 
     hsplit = optional(host_split)
 
@@ -396,7 +426,7 @@ def run_ours(args, rank, world, dist):
             qkv_h, keep_h, cls_h = host_in[(c, i)]
             pl.dense_qkv.copy_(qkv_h, non_blocking=True)
             pl.keep.copy_(keep_h, non_blocking=True)
-            pl.replay()
+            pl.launch(sync=False)
             cls_h.copy_(pl.cls_out, non_blocking=True)
             stream.synchronize()
 
@@ -575,9 +605,11 @@ def run_ours(args, rank, world, dist):
           "config": {"workload": "serving_deit_s_b1-4_p0-80", "B": list(synthetic.SERVING_BATCHES),
                      "prune_rates": list(synthetic.SERVING_RATES), "jitter": 0.10, "L_full": 197,
                      "heads": 6, "head_dim": 64, "calls_per_step": len(CASES),
-                     "call": "Pipeline.replay(): CUDA graph of ragged_pipeline in fused mode (one kernel: pack, "
-                             "attention, CLS), then stream synchronize; direct_call_us_per_call = the same "
-                             "pipeline as one C call that waits for completion (RAGGED_PIPELINE_SYNC)",
+                     "call": "Pipeline.launch(sync=True): one call into libragged that launches its CUDA graph "
+                             "of ragged_pipeline in fused mode (one kernel: pack, attention, CLS) and waits "
+                             "for it; torch_graph_us_per_call = torch's graph of the same call, replay + stream "
+                             "synchronize; direct_call_us_per_call = the pipeline as one C call that enqueues "
+                             "and waits (RAGGED_PIPELINE_SYNC)",
                      "l2": f"inputs rotated over {ncopies} copies ({ncopies * per_copy / 2**20:.0f} MiB > 2x L2)",
                      "parallelism": "replicas" if world > 1 else "single"},
           "e2e": {"value": round(e2e_us, 3), "unit": "µs/call", "h2d_bytes_per_step": int(h2d),
@@ -585,6 +617,7 @@ def run_ours(args, rank, world, dist):
           "gpu_launches": gpu_launches,
           "roofline": roofline,
           "direct_call_us_per_call": round(direct_us, 3),
+          "torch_graph_us_per_call": round(torch_graph_us, 3),
           "warm_us_per_call": round(warm_us, 3),
           "per_case": detail,
           "host_split": hsplit,

@@ -335,6 +335,39 @@ RAGGED_API ragged_status ragged_pipeline_noalloc(const void *dense_qkv, const ui
                                                  void *cls_out, void *stream);
 
 /*
+ * A pipeline call recorded once as a CUDA graph that the library owns, so that
+ * each later call is one graph launch, and with RAGGED_PIPELINE_SYNC the wait
+ * for it too, in a single call.  Paper: radpulse section "Bypassing the
+ * binding" and its section on the FA2 dispatch ceiling (the fixed host cost of
+ * a varlen call is argument handling, allocation and the launch path; here a
+ * call is one crossing into this library and one graph launch).
+ *
+ * ragged_pipeline_graph_create records ragged_pipeline with these arguments
+ * (flags without RAGGED_PIPELINE_SYNC) on `stream`, which must be a created
+ * stream, not the legacy default one.  It first runs the call once outside
+ * the recording (so it validates the arguments and does the per-device set-up;
+ * the outputs are written), then records it and instantiates the graph.  The
+ * graph objects are allocated here, once.  Every launch reads and writes the
+ * same buffers, with the same sizes; the buffers must stay valid until the
+ * graph is destroyed.  *graph_out is NULL on failure.
+ *
+ * ragged_pipeline_graph_launch launches it on `stream` (any stream of the same
+ * device); flags is 0 or RAGGED_PIPELINE_SYNC, which also waits for it
+ * (cudaStreamSynchronize) before returning.  Launching allocates nothing.
+ *
+ * ragged_pipeline_graph_destroy frees the graph (NULL is a no-op).
+ */
+typedef struct ragged_pipeline_graph ragged_pipeline_graph;
+
+RAGGED_API ragged_status ragged_pipeline_graph_create(const void *dense_qkv, const uint8_t *keep, int64_t B,
+                                                      int64_t L_full, int64_t H, int64_t head_dim, float scale,
+                                                      ragged_dtype dtype, void *packed_qkv, int32_t *cu_seqlens,
+                                                      void *out, void *cls_out, uint32_t flags, void *stream,
+                                                      ragged_pipeline_graph **graph_out);
+RAGGED_API ragged_status ragged_pipeline_graph_launch(ragged_pipeline_graph *graph, void *stream, uint32_t flags);
+RAGGED_API ragged_status ragged_pipeline_graph_destroy(ragged_pipeline_graph *graph);
+
+/*
  * ragged_get_device_status - read and clear the status word of the current
  * device.  Synchronises with `stream` (the only call that does).  *host_out
  * receives the RAGGED_DEV_* bits set since the previous read.

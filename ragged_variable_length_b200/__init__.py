@@ -56,7 +56,8 @@ DTYPE_NAMES = {"f16": torch.float16, "bf16": torch.bfloat16, "f32": torch.float3
 EXPORTS = ("ragged_pack", "ragged_attn_fwd", "ragged_unpack_cls", "ragged_unpack",
            "ragged_pipeline", "ragged_get_device_status", "ragged_status_string",
            "ragged_last_error", "ragged_abi_version", "ragged_set_attn_kernel",
-           "ragged_mask_l2", "ragged_pack_topk", "ragged_pipeline_noalloc")
+           "ragged_mask_l2", "ragged_pack_topk", "ragged_pipeline_noalloc", "ragged_pipeline_graph_create",
+           "ragged_pipeline_graph_launch", "ragged_pipeline_graph_destroy")
 
 
 class RaggedError(RuntimeError):
@@ -86,9 +87,14 @@ def load(path: Optional[str] = None):
     lib.ragged_unpack.argtypes = [vp, vp, vp, i64, i64, i64, vp, vp]
     lib.ragged_pipeline.argtypes = [vp, vp, i64, i64, i64, i64, f32, i32, vp, vp, vp, vp, ctypes.c_uint32, vp]
     lib.ragged_pipeline_noalloc.argtypes = [vp, vp, i64, i64, i64, i64, f32, i32, vp, vp, vp, vp]
+    lib.ragged_pipeline_graph_create.argtypes = [vp, vp, i64, i64, i64, i64, f32, i32, vp, vp, vp, vp,
+                                                 ctypes.c_uint32, vp, ctypes.POINTER(vp)]
+    lib.ragged_pipeline_graph_launch.argtypes = [vp, vp, ctypes.c_uint32]
+    lib.ragged_pipeline_graph_destroy.argtypes = [vp]
     lib.ragged_get_device_status.argtypes = [ctypes.POINTER(ctypes.c_uint32), vp]
     for name in ("ragged_pack", "ragged_attn_fwd", "ragged_unpack_cls", "ragged_unpack",
-                 "ragged_pipeline", "ragged_get_device_status", "ragged_pipeline_noalloc"):
+                 "ragged_pipeline", "ragged_get_device_status", "ragged_pipeline_noalloc",
+                 "ragged_pipeline_graph_create", "ragged_pipeline_graph_launch", "ragged_pipeline_graph_destroy"):
         getattr(lib, name).restype = ctypes.c_int
     lib.ragged_status_string.argtypes = [ctypes.c_int]
     lib.ragged_status_string.restype = ctypes.c_char_p
@@ -314,6 +320,11 @@ class _PipelineArgs(ctypes.Structure):
                 ("flags", ctypes.c_uint32), ("stream", ctypes.c_void_p)]
 
 
+class _GraphArgs(ctypes.Structure):
+    """The parameters of ragged_pipeline_graph_launch (argument block of _fastcall.graph_run)."""
+    _fields_ = [("graph", ctypes.c_void_p), ("stream", ctypes.c_void_p), ("flags", ctypes.c_uint32)]
+
+
 _fast = None
 
 
@@ -330,6 +341,9 @@ def _fast_forwarder():
         if fc.args_size() != ctypes.sizeof(_PipelineArgs):
             raise RuntimeError("_fastcall argument block does not match the binding")
         fc.bind(ctypes.cast(load().ragged_pipeline, ctypes.c_void_p).value)
+        if fc.graph_args_size() != ctypes.sizeof(_GraphArgs):
+            raise RuntimeError("_fastcall graph argument block does not match the binding")
+        fc.bind_graph(ctypes.cast(load().ragged_pipeline_graph_launch, ctypes.c_void_p).value)
         _fast = fc
     return _fast or None
 
@@ -404,6 +418,46 @@ class Pipeline:
         torch.cuda.current_stream().wait_stream(s)
         self.bind_inputs(*self._inputs)
         self.graph = g
+
+    def record(self, stream=None) -> None:
+        """Record the pipeline as a CUDA graph that libragged owns
+        (ragged_pipeline_graph_create); launch() then costs one crossing into
+        the library: one graph launch, and with sync=True the wait for it."""
+        lib = load()
+        strm = _stream(stream)
+        a = self._args
+        handle = ctypes.c_void_p()
+        _check(lib.ragged_pipeline_graph_create(a[0], a[1], a[2], a[3], a[4], a[5], a[6], a[7], a[8], a[9],
+                                                a[10], a[11], ctypes.c_uint32(self.flags), ctypes.c_void_p(strm),
+                                                ctypes.byref(handle)))
+        self.release()
+        self._graph_handle = handle
+        self._graph_block = _GraphArgs(handle.value, strm, RAGGED_PIPELINE_SYNC)
+        self._graph_block_async = _GraphArgs(handle.value, strm, 0)
+        self._graph_block_addr = ctypes.addressof(self._graph_block)
+        self._graph_block_async_addr = ctypes.addressof(self._graph_block_async)
+
+    def launch(self, sync: bool = True) -> None:
+        """Launch the graph recorded by record(); with sync=True, return once it has finished."""
+        addr = self._graph_block_addr if sync else self._graph_block_async_addr
+        st = self._fc.graph_run(addr) if self._fc else \
+            load().ragged_pipeline_graph_launch(self._graph_handle, ctypes.c_void_p(self._graph_block.stream),
+                                                ctypes.c_uint32(self._graph_block.flags if sync else 0))
+        if st:
+            _check(st)
+
+    def release(self) -> None:
+        """Free the graph recorded by record(), if any."""
+        h = getattr(self, "_graph_handle", None)
+        if h is not None and h.value:
+            load().ragged_pipeline_graph_destroy(h)
+        self._graph_handle = None
+
+    def __del__(self):
+        try:
+            self.release()
+        except Exception:  # noqa: BLE001 - interpreter shutdown
+            pass
 
     def replay(self) -> None:
         self.graph.replay()

@@ -1,6 +1,8 @@
 /*
  * _fastcall: a CPython extension that forwards one pre-marshalled
- * ragged_pipeline call to the C ABI in a single Python -> C crossing.
+ * ragged_pipeline call, or one launch of a recorded pipeline graph
+ * (ragged_pipeline_graph_launch), to the C ABI in a single Python -> C
+ * crossing.
  *
  * The Python binding builds the argument block (struct pipeline_args, the
  * parameters of ragged_pipeline in order) once per buffer set and passes its
@@ -31,6 +33,16 @@ typedef struct {
 } pipeline_args;
 
 static pipeline_fn g_pipeline = NULL;
+
+typedef int (*graph_launch_fn)(void *, void *, uint32_t);
+
+typedef struct {
+    void *graph;
+    void *stream;
+    uint32_t flags;
+} graph_args;
+
+static graph_launch_fn g_graph_launch = NULL;
 
 static PyObject *fc_bind(PyObject *self, PyObject *arg)
 {
@@ -63,6 +75,43 @@ static PyObject *fc_run(PyObject *self, PyObject *arg)
     return PyLong_FromLong(status);
 }
 
+static PyObject *fc_bind_graph(PyObject *self, PyObject *arg)
+{
+    (void)self;
+    void *p = PyLong_AsVoidPtr(arg);
+    if (p == NULL && PyErr_Occurred())
+        return NULL;
+    g_graph_launch = (graph_launch_fn)p;
+    Py_RETURN_NONE;
+}
+
+static PyObject *fc_graph_run(PyObject *self, PyObject *arg)
+{
+    (void)self;
+    const graph_args *a = (const graph_args *)PyLong_AsVoidPtr(arg);
+    if (a == NULL) {
+        if (!PyErr_Occurred())
+            PyErr_SetString(PyExc_ValueError, "null argument block");
+        return NULL;
+    }
+    if (g_graph_launch == NULL) {
+        PyErr_SetString(PyExc_RuntimeError, "ragged_pipeline_graph_launch is not bound");
+        return NULL;
+    }
+    int status;
+    Py_BEGIN_ALLOW_THREADS
+    status = g_graph_launch(a->graph, a->stream, a->flags);
+    Py_END_ALLOW_THREADS
+    return PyLong_FromLong(status);
+}
+
+static PyObject *fc_graph_args_size(PyObject *self, PyObject *unused)
+{
+    (void)self;
+    (void)unused;
+    return PyLong_FromSize_t(sizeof(graph_args));
+}
+
 static PyObject *fc_args_size(PyObject *self, PyObject *unused)
 {
     (void)self;
@@ -74,6 +123,9 @@ static PyMethodDef fc_methods[] = {
     {"bind", fc_bind, METH_O, "bind(address of ragged_pipeline)"},
     {"run", fc_run, METH_O, "run(address of a pipeline argument block) -> ragged_status"},
     {"args_size", fc_args_size, METH_NOARGS, "size in bytes of the argument block"},
+    {"bind_graph", fc_bind_graph, METH_O, "bind(address of ragged_pipeline_graph_launch)"},
+    {"graph_run", fc_graph_run, METH_O, "graph_run(address of a graph argument block) -> ragged_status"},
+    {"graph_args_size", fc_graph_args_size, METH_NOARGS, "size in bytes of the graph argument block"},
     {NULL, NULL, 0, NULL},
 };
 

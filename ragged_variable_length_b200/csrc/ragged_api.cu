@@ -18,6 +18,7 @@
 #include <atomic>
 #include <cudaTypedefs.h>
 #include <mutex>
+#include <new>
 #include "common.cuh"
 #include "mask.cuh"
 #include "pack.cuh"
@@ -701,5 +702,73 @@ RAGGED_API ragged_status ragged_test_set_hooks(int32_t hook, uint32_t spin_limit
                       "test spin limit");
 }
 #endif
+
+// ---- library-owned CUDA graph of one pipeline call -------------------------
+
+struct ragged_pipeline_graph {
+    cudaGraph_t graph;
+    cudaGraphExec_t exec;
+    int device;
+};
+
+ragged_status ragged_pipeline_graph_create(const void* dense_qkv, const uint8_t* keep, int64_t B, int64_t L_full,
+                                           int64_t H, int64_t head_dim, float scale, ragged_dtype dtype,
+                                           void* packed_qkv, int32_t* cu_seqlens, void* out, void* cls_out,
+                                           uint32_t flags, void* stream, ragged_pipeline_graph** graph_out) {
+    if (graph_out == nullptr) return fail(RAGGED_ERR_INVALID_ARG, "graph_out is NULL");
+    *graph_out = nullptr;
+    if (flags & RAGGED_PIPELINE_SYNC) return fail(RAGGED_ERR_INVALID_ARG, "RAGGED_PIPELINE_SYNC cannot be recorded");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (s == nullptr) return fail(RAGGED_ERR_INVALID_ARG, "a graph is recorded on a created stream, not the default one");
+    // One call outside the capture: argument checks, and the per-device
+    // set-up (kernel attributes, tensor maps) that must not be recorded.
+    ragged_status st = ragged_pipeline(dense_qkv, keep, B, L_full, H, head_dim, scale, dtype, packed_qkv, cu_seqlens,
+                                       out, cls_out, flags, stream);
+    if (st != RAGGED_OK) return st;
+    int dev = 0;
+    st = cuda_check(cudaGetDevice(&dev), "cudaGetDevice");
+    if (st != RAGGED_OK) return st;
+    st = cuda_check(cudaStreamBeginCapture(s, cudaStreamCaptureModeThreadLocal), "cudaStreamBeginCapture");
+    if (st != RAGGED_OK) return st;
+    const ragged_status call = ragged_pipeline(dense_qkv, keep, B, L_full, H, head_dim, scale, dtype, packed_qkv,
+                                               cu_seqlens, out, cls_out, flags, stream);
+    cudaGraph_t graph = nullptr;
+    st = cuda_check(cudaStreamEndCapture(s, &graph), "cudaStreamEndCapture");
+    if (call != RAGGED_OK || st != RAGGED_OK) {
+        if (graph != nullptr) cudaGraphDestroy(graph);
+        return call != RAGGED_OK ? call : st;
+    }
+    cudaGraphExec_t exec = nullptr;
+    st = cuda_check(cudaGraphInstantiate(&exec, graph, 0), "cudaGraphInstantiate");
+    if (st != RAGGED_OK) {
+        cudaGraphDestroy(graph);
+        return st;
+    }
+    ragged_pipeline_graph* g = new (std::nothrow) ragged_pipeline_graph{graph, exec, dev};
+    if (g == nullptr) {
+        cudaGraphExecDestroy(exec);
+        cudaGraphDestroy(graph);
+        return fail(RAGGED_ERR_CUDA, "out of host memory");
+    }
+    *graph_out = g;
+    return RAGGED_OK;
+}
+
+ragged_status ragged_pipeline_graph_launch(ragged_pipeline_graph* graph, void* stream, uint32_t flags) {
+    if (graph == nullptr) return fail(RAGGED_ERR_INVALID_ARG, "graph is NULL");
+    if ((flags & ~RAGGED_PIPELINE_SYNC) != 0) return fail(RAGGED_ERR_INVALID_ARG, "flags = %u", flags);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    ragged_status st = cuda_check(cudaGraphLaunch(graph->exec, s), "cudaGraphLaunch");
+    if (st != RAGGED_OK || !(flags & RAGGED_PIPELINE_SYNC)) return st;
+    return cuda_check(cudaStreamSynchronize(s), "cudaStreamSynchronize");
+}
+
+ragged_status ragged_pipeline_graph_destroy(ragged_pipeline_graph* graph) {
+    if (graph == nullptr) return RAGGED_OK;
+    ragged_status st = cuda_check(cudaGraphExecDestroy(graph->exec), "cudaGraphExecDestroy");
+    const ragged_status st2 = cuda_check(cudaGraphDestroy(graph->graph), "cudaGraphDestroy");
+    delete graph;
+    return st != RAGGED_OK ? st : st2;
+}
 
 }  // extern "C"

@@ -222,3 +222,19 @@ def test_test_hooks_live_only_in_the_test_build():
     assert re.search(r" T ragged_test_set_hooks\b", test)
     header = open(os.path.join(ROOT, "include", "ragged_test_hooks.h")).read()
     assert "RAGGED_API ragged_status ragged_test_set_hooks(" in header
+
+
+def test_pipeline_graph_rejects_bad_arguments(lib):
+    """ragged_pipeline_graph_*: argument errors come back before any CUDA call."""
+    out = ctypes.c_void_p(123)
+    args = (A16, A16, 4, 197, 6, 64, ctypes.c_float(0.125), rv.RAGGED_F16, None, A16, A16, None)
+    assert lib.ragged_pipeline_graph_create(*args, rv.RAGGED_PIPELINE_FUSED, A16, None) == rv.RAGGED_ERR_INVALID_ARG
+    assert "graph_out" in rv.ragged_last_error()
+    assert lib.ragged_pipeline_graph_create(*args, rv.RAGGED_PIPELINE_SYNC, A16,
+                                            ctypes.byref(out)) == rv.RAGGED_ERR_INVALID_ARG
+    assert out.value is None and "SYNC" in rv.ragged_last_error()
+    assert lib.ragged_pipeline_graph_create(*args, 0, None, ctypes.byref(out)) == rv.RAGGED_ERR_INVALID_ARG
+    assert "default" in rv.ragged_last_error()
+    assert lib.ragged_pipeline_graph_launch(None, None, 0) == rv.RAGGED_ERR_INVALID_ARG
+    assert lib.ragged_pipeline_graph_launch(A16, None, 8) == rv.RAGGED_ERR_INVALID_ARG
+    assert lib.ragged_pipeline_graph_destroy(None) == rv.RAGGED_OK

@@ -137,3 +137,28 @@ def test_run_sync_matches_enqueue_then_sync(flags):
     assert torch.equal(p.cls_out, cls_ref)
     packed_o, cu_o = oracle.pack(w.qkv, w.keep)
     assert np.array_equal(p.cu_seqlens.cpu().numpy(), cu_o)
+
+
+def test_recorded_graph_matches_the_direct_call():
+    """ragged_pipeline_graph_create / _launch: the recorded pipeline gives what
+    ragged_pipeline gives, and picks up new inputs written into its buffers."""
+    w = synthetic.serving(4, 0.5)
+    p = rv.Pipeline(w.B, w.L_full, w.H, torch.float16, flags=rv.RAGGED_PIPELINE_FUSED)
+    s = torch.cuda.Stream()
+    p.dense_qkv.copy_(to_device(w.qkv, "f16"))
+    p.keep.copy_(torch.from_numpy(w.keep))
+    torch.cuda.synchronize()
+    p.bind_inputs(p.dense_qkv, p.keep, stream=s)
+    p.record(stream=s)
+    for wk in (w, synthetic.serving(4, 0.5, copy=1)):
+        p.dense_qkv.copy_(to_device(wk.qkv, "f16"))
+        p.keep.copy_(torch.from_numpy(wk.keep))
+        torch.cuda.synchronize()
+        p.cls_out.zero_()
+        p.launch(sync=True)
+        _, cu_ref, out_ref, cls_ref = run(wk, rv.RAGGED_PIPELINE_FUSED, materialize_packed=False)
+        T = int(cu_ref[-1].item())
+        assert torch.equal(p.cu_seqlens, cu_ref)
+        assert torch.equal(p.out[:T], out_ref[:T]) and torch.equal(p.cls_out, cls_ref)
+    p.release()
+    assert rv.ragged_get_device_status() == 0
