@@ -154,7 +154,9 @@ RAGGED_API ragged_status ragged_attn_fwd(const void *q, const void *k, const voi
 #define RAGGED_ATTN_TCGEN05 3    /* tcgen05.mma with TMEM accumulators, K/V streamed, one
                                     CTA per (128-query tile, head, sequence)               */
 #define RAGGED_ATTN_PERSISTENT 4 /* tcgen05.mma, persistent CTAs with a TMA load warp;
-                                    B <= 1024 (larger B runs RAGGED_ATTN_TCGEN05)          */
+                                    B <= 1024, H <= 1023, max_seqlen <= 2047 * 128 and
+                                    B * H * ceil(max_seqlen / 128) at most 1024 items per
+                                    CTA (two CTAs per SM); otherwise RAGGED_ATTN_TCGEN05   */
 
 /*
  * ragged_set_attn_kernel - process-wide choice of the f16/bf16 attention

@@ -9,13 +9,14 @@
 //
 // Work items are (sequence, 128-query tile, head) triples, numbered densely.
 // Each CTA copies cu_seqlens into shared memory once, forms the exclusive
-// prefix of H * ceil(L_b / 128) over the sequences, and takes items
-// blockIdx.x, blockIdx.x + gridDim.x, ...; two CTAs share an SM.  TMEM
-// (256 columns: S of two tiles, each overwritten in place by its P, and two
-// O buffers for alternate items) and the mbarriers are set up once per CTA,
-// so the per-launch fixed costs of a CTA (cu_seqlens read, TMEM allocation,
-// first loads) are paid once, and the loads of the next item run under the
-// softmax of the current one.
+// prefix of H * ceil(L_b / 128) over the sequences, and decodes its own items
+// (blockIdx.x, blockIdx.x + gridDim.x, ...) once into a list of packed words,
+// so that each role reads its next item with one shared-memory load; two CTAs
+// share an SM.  TMEM (256 columns: S of three tiles, each overwritten in
+// place by its P, and O) and the mbarriers are set up once per CTA, so the
+// per-launch fixed costs of a CTA (cu_seqlens read, TMEM allocation, first
+// loads) are paid once, and the loads of the next item run under the softmax
+// of the current one.
 //
 // Warp roles; they hand off through mbarriers only:
 //   warp 5     loads.  Full tiles by TMA from 3-D tensor maps over
@@ -23,23 +24,22 @@
 //              canonical SWIZZLE_128B operand layout of tcgen05; partial tiles
 //              (the last rows of a sequence) by cp.async with zero fill, each
 //              lane's arrival triggered by the completion of its copies
-//              (cp.async.mbarrier.arrive.noinc).  Q is double-buffered, K/V
-//              flow through a 4-stage ring; the stage of an item's last tile
-//              is handed back by the softmax warps once the epilogue has used
-//              it to stage O for row-contiguous stores.
-//   warp 4     one thread issues every tcgen05.mma.  Q K^T runs two tiles
+//              (cp.async.mbarrier.arrive.noinc).  Q is double-buffered; K and
+//              V flow through separate rings (3 and 5 stages), each stage
+//              handed back by the completion of the product that read it.
+//   warp 4     one thread issues every tcgen05.mma.  Q K^T runs three tiles
 //              ahead of P V: P V(g) as soon as P(g) is in TMEM, then S of tile
-//              g + 2 into TMEM buffer g & 1 (in order behind P V(g), which
+//              g + 3 into TMEM buffer g % 3 (in order behind P V(g), which
 //              read P(g) from it).  Across items the walks simply continue.
 //   warps 0-3  softmax, one thread per query row (TMEM lane = row), single
 //              pass with a reference maximum that is raised (and the running
 //              sum and O rescaled) only when a tile exceeds it by more than
 //              2^8; P (bf16: hi and lo parts) replaces S in its TMEM buffer.
 //              The pairwise fp32 work uses the packed f32x2 instructions of
-//              sm_100.  An item's epilogue (O / l and the CLS row) runs after
-//              the first tile of the next item, from the item's own O buffer,
-//              so the softmax warps never wait at an item boundary for the
-//              last product.
+//              sm_100.  An item's epilogue (O / l and the CLS row) runs at the
+//              first tile of the next item, before that tile's P is handed
+//              over (its product overwrites O): each thread reads its row of
+//              O from TMEM and stores it with 32-byte stores.
 // The tile counter g runs across items, so every buffer parity carries over
 // from one item to the next.
 //
@@ -56,20 +56,32 @@ namespace ragged {
 namespace tc05 {
 
 constexpr int kPersistThreads = 192;
-constexpr int kPersistStages = 4;
-// TMEM per CTA (256 columns): S of two tiles at [0, 64) and [64, 128), each
-// overwritten in place by its P (16-bit pairs; bf16 as hi + lo halves), and
-// two O buffers at [128, 192) and [192, 256), one per alternate item.
-constexpr uint32_t kOBufCol = 128;
+// TMEM per CTA (256 columns): S of three tiles at [0, 64), [64, 128) and
+// [128, 192), each overwritten in place by its P (16-bit pairs; bf16 as hi +
+// lo halves), and O at [192, 256).
+constexpr int kSBufs = 3;
+// K tiles are read once, by the Q K^T of their tile, and V tiles by its P V,
+// kSBufs tiles later: K and V flow through separate rings.  K stage g % kSBufs
+// is refilled once the Q K^T of tile g - kSBufs has finished, which the scores
+// barrier of the same index reports (its next phase needs the new K tile, so
+// a parity wait on it is exact); V stage g % 5 once the P V of tile g - 5 has.
+constexpr int kKStages = kSBufs;
+constexpr int kVStages = 5;
+constexpr uint32_t kOCol = kSBufs * 64;
 constexpr int kPersistMaxB = 1024;   // cu_seqlens and item offsets live in shared memory
+// Each CTA decodes its own work items once, into shared memory (one packed
+// word each: sequence, head, query tile), so that every role reads an item
+// with a single shared-memory load instead of a binary search.
+constexpr int kPersistMaxItems = 1024;
 constexpr int kMmaWarp = 4;
 constexpr int kLoadWarp = 5;
 constexpr uint32_t kFullMask = 0xffffffffu;
 
-// Dynamic shared memory: alignment slack, two Q buffers, the K/V ring, then
-// cu_seqlens and the item offsets (B + 1 ints each).
-__host__ __device__ constexpr int persist_smem_bytes(int B) {
-    return 1024 + 2 * kQBytes + kPersistStages * 2 * kKVTileBytes + 2 * (B + 1) * 4;
+// Dynamic shared memory: alignment slack, two Q buffers, the K ring, the V
+// ring, cu_seqlens and the item offsets (B + 1 ints each), then the CTA's
+// item list (items_cap words).
+__host__ __device__ constexpr int persist_smem_bytes(int B, int items_cap) {
+    return 1024 + 2 * kQBytes + (kKStages + kVStages) * kKVTileBytes + 2 * (B + 1) * 4 + items_cap * 4;
 }
 
 struct PersistArgs {
@@ -83,6 +95,7 @@ struct PersistArgs {
     uint16_t* out;
     int64_t out_tok_stride;
     uint16_t* cls_out;
+    int items_cap;   // at least the number of items of any CTA
 };
 
 // ---- mbarrier, TMA and packed-fp32 wrappers --------------------------------
@@ -212,26 +225,39 @@ __device__ __forceinline__ Item decode_item(int j, const int* s_cu, const int* s
     return it;
 }
 
-// Cursor over the tiles of a CTA's items: item j (the k-th of this CTA),
-// key tile t of it.
+// An item packed into one word: sequence (11 bits), head (10), query tile (11).
+__device__ __forceinline__ uint32_t pack_item(const Item& it) {
+    return static_cast<uint32_t>(it.b) | (static_cast<uint32_t>(it.h) << 11) |
+           (static_cast<uint32_t>(it.q0 / kRows) << 21);
+}
+__device__ __forceinline__ Item unpack_item(uint32_t w, const int* s_cu) {
+    Item it;
+    it.b = static_cast<int>(w & 2047u);
+    it.h = static_cast<int>((w >> 11) & 1023u);
+    it.q0 = static_cast<int>(w >> 21) * kRows;
+    it.start = s_cu[it.b];
+    it.len = s_cu[it.b + 1] - it.start;
+    it.nt = (it.len + kTileN - 1) / kTileN;
+    return it;
+}
+
+// Cursor over the tiles of a CTA's items: its k-th item, key tile t of it.
 struct Walk {
-    int j, k, t, total;
+    int k, t, n;
     bool valid;
     Item it;
+    const uint32_t* items;
     const int* s_cu;
-    const int* s_ip;
-    int B, H;
-    __device__ __forceinline__ Walk(int j0, int total_, const int* cu, const int* ip, int B_, int H_)
-        : j(j0), k(0), t(0), total(total_), valid(j0 < total_), s_cu(cu), s_ip(ip), B(B_), H(H_) {
-        if (valid) it = decode_item(j, s_cu, s_ip, B, H);
+    __device__ __forceinline__ Walk(int n_, const uint32_t* items_, const int* cu)
+        : k(0), t(0), n(n_), valid(n_ > 0), items(items_), s_cu(cu) {
+        if (valid) it = unpack_item(items[0], s_cu);
     }
     __device__ __forceinline__ void next() {
         if (++t < it.nt) return;
         t = 0;
         ++k;
-        j += gridDim.x;
-        valid = j < total;
-        if (valid) it = decode_item(j, s_cu, s_ip, B, H);
+        valid = k < n;
+        if (valid) it = unpack_item(items[k], s_cu);
     }
 };
 
@@ -240,62 +266,51 @@ __global__ void __launch_bounds__(kPersistThreads, 2)
     attn_tc05_persist_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                              const __grid_constant__ CUtensorMap tm_v, const PersistArgs a) {
     extern __shared__ uint8_t smem_raw[];
-    // kv_full[S], kv_empty[S], q_full[2], q_empty[2], s_full[2], p_full[0..1], pv_done[2], o_empty[0], drain,
-    // o_empty[1], (unused), p_full[2..3], o_staged, o_stored
-    __shared__ __align__(8) uint64_t s_bar[2 * kPersistStages + 18];
+    // kv_full[3], q_full[2], q_empty[2], s_full[kSBufs], p_full[4], pv_done[5], drain
+    __shared__ __align__(8) uint64_t s_bar[17 + kSBufs];
     __shared__ uint32_t s_tmem;
     __shared__ int s_fail;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    constexpr int S = kPersistStages;
     constexpr int kParts = Cvt<T>::kParts;
 
     const uint32_t raw = smem_addr(smem_raw);
-    const uint32_t sQ = (raw + 1023u) & ~1023u;   // Q buffer i at sQ + i * 16 KB
-    const uint32_t sRing = sQ + 2 * kQBytes;      // stage s: K at sRing + s * 16 KB, V 8 KB further
-    int* s_cu = reinterpret_cast<int*>(smem_raw + (sRing - raw) + S * 2 * kKVTileBytes);
+    const uint32_t sQ = (raw + 1023u) & ~1023u;     // Q buffer i at sQ + i * 16 KB
+    const uint32_t sK = sQ + 2 * kQBytes;           // K stage s at sK + s * 8 KB
+    const uint32_t sV = sK + kKStages * kKVTileBytes;   // V stage s at sV + s * 8 KB
+    int* s_cu = reinterpret_cast<int*>(smem_raw + (sV - raw) + kVStages * kKVTileBytes);
     int* s_ip = s_cu + (a.B + 1);
+    uint32_t* s_items = reinterpret_cast<uint32_t*>(s_ip + (a.B + 1));
 
     const uint32_t bar0 = smem_addr(&s_bar[0]);
-    auto kv_full = [&](int s) { return bar0 + 8u * s; };
-    auto kv_empty = [&](int s) { return bar0 + 8u * (S + s); };
-    auto q_full = [&](int i) { return bar0 + 8u * (2 * S + i); };
-    auto q_empty = [&](int i) { return bar0 + 8u * (2 * S + 2 + i); };
-    auto s_full = [&](int i) { return bar0 + 8u * (2 * S + 4 + i); };
-    // P of tile g is signalled on p_full(g & 3): warps with no rows in the
-    // current query tile skip the softmax and may arrive for tile g + 2 while
-    // another warp is still working on tile g, so tiles two apart must not
-    // share a barrier (three tiles apart is impossible: Q K^T of tile g + 3
-    // waits until every warp has read S(g + 1)).
-    auto p_full = [&](int i) { return bar0 + 8u * (i < 2 ? 2 * S + 6 + i : 2 * S + 14 + (i - 2)); };
-    auto pv_done = [&](int i) { return bar0 + 8u * (2 * S + 8 + i); };
-    // O buffer i has been read out by the epilogue of its item.
-    auto o_empty = [&](int i) { return bar0 + 8u * (i == 0 ? 2 * S + 10 : 2 * S + 12); };
-    const uint32_t drain = bar0 + 8u * (2 * S + 11);
-    // The epilogue's O tile is staged in shared memory / has been stored
-    // (128 arrivals each, one phase per item).
-    const uint32_t o_staged = bar0 + 8u * (2 * S + 16);
-    const uint32_t o_stored = bar0 + 8u * (2 * S + 17);
+    // K and V of tile g have landed (g % 3; a K stage is refilled only after the
+    // Q K^T that read it, so a tile three ahead cannot reach the barrier first).
+    auto kv_full = [&](int i) { return bar0 + 8u * i; };
+    auto q_full = [&](int i) { return bar0 + 8u * (3 + i); };
+    auto q_empty = [&](int i) { return bar0 + 8u * (5 + i); };
+    // S of tile g is in TMEM buffer g % 3; the same completion frees K stage g % 3.
+    auto s_full = [&](int i) { return bar0 + 8u * (7 + i); };
+    // P of tile g is in TMEM (g & 3): warps with no rows in the current query
+    // tile skip the softmax and can run up to three tiles ahead of a warp
+    // that has rows (Q K^T of tile g waits for P of tile g - 3), so four tiles
+    // in a row must not share a barrier.
+    auto p_full = [&](int i) { return bar0 + 8u * (7 + kSBufs + i); };
+    // P V of tile g has finished (g % 5); the same completion frees V stage g % 5.
+    auto pv_done = [&](int i) { return bar0 + 8u * (11 + kSBufs + i); };
+    const uint32_t drain = bar0 + 8u * (16 + kSBufs);
     volatile int* fail_flag = &s_fail;
 
     // ---- setup: cu_seqlens, barriers, TMEM, item offsets ----
     for (int i = tid; i <= a.B; i += kPersistThreads) s_cu[i] = __ldg(a.cu + i);
     if (tid == 0) {
-        for (int s = 0; s < S; ++s) {
-            mbar_init(kv_full(s), 32);
-            mbar_init(kv_empty(s), 1);
-        }
+        for (int i = 0; i < 3; ++i) mbar_init(kv_full(i), 32);
+        for (int i = 0; i < kSBufs; ++i) mbar_init(s_full(i), 1);
         for (int i = 0; i < 2; ++i) {
             mbar_init(q_full(i), 32);
             mbar_init(q_empty(i), 1);
-            mbar_init(s_full(i), 1);
-            mbar_init(p_full(i), kSoftmaxThreads);
-            mbar_init(p_full(i + 2), kSoftmaxThreads);
-            mbar_init(pv_done(i), 1);
-            mbar_init(o_empty(i), kSoftmaxThreads);
         }
-        mbar_init(o_staged, kSoftmaxThreads);
-        mbar_init(o_stored, kSoftmaxThreads);
+        for (int i = 0; i < 4; ++i) mbar_init(p_full(i), kSoftmaxThreads);
+        for (int i = 0; i < 5; ++i) mbar_init(pv_done(i), 1);
         mbar_init(drain, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         s_fail = 0;
@@ -340,7 +355,17 @@ __global__ void __launch_bounds__(kPersistThreads, 2)
         }
     }
     __syncthreads();
+    // This CTA's items (blockIdx.x, blockIdx.x + gridDim.x, ...), decoded once.
     const int total = s_ip[a.B];
+    int n_items = static_cast<int>(blockIdx.x) < total ? (total - 1 - static_cast<int>(blockIdx.x)) / static_cast<int>(gridDim.x) + 1 : 0;
+    if (n_items > a.items_cap) {   // the host sizes items_cap from B, H and max_seqlen; never reached
+        if (tid == 0) raise_status(RAGGED_DEV_BAD_SEQLENS);
+        n_items = 0;
+    }
+    for (int k = tid; k < n_items; k += kPersistThreads)
+        s_items[k] = pack_item(decode_item(static_cast<int>(blockIdx.x) + k * static_cast<int>(gridDim.x), s_cu, s_ip,
+                                           a.B, a.H));
+    __syncthreads();
     const uint32_t tmem = s_tmem;
 
     if (warp == kLoadWarp) {
@@ -360,9 +385,9 @@ __global__ void __launch_bounds__(kPersistThreads, 2)
         uint32_t g = 0;
         int k = 0;
         bool ok = !test_hook(1);
-        for (int j = blockIdx.x; ok && j < total; j += gridDim.x, ++k) {
+        for (; ok && k < n_items; ++k) {
             if (__any_sync(kFullMask, *fail_flag != 0)) break;
-            const Item it = decode_item(j, s_cu, s_ip, a.B, a.H);
+            const Item it = unpack_item(s_items[k], s_cu);
             const int64_t seq_off = static_cast<int64_t>(it.start) * a.tok_stride +
                                     static_cast<int64_t>(it.h) * a.head_stride;
             const int qb = k & 1;
@@ -380,33 +405,43 @@ __global__ void __launch_bounds__(kPersistThreads, 2)
                 publish_copies(q_full(qb));
             }
             for (int t = 0; t < it.nt; ++t, ++g) {
-                const int s = static_cast<int>(g % S);
-                if (g >= static_cast<uint32_t>(S) && !warp_wait(kv_empty(s), ((g / S) - 1) & 1)) {
+                // K stage g % 3 is free once the Q K^T of tile g - 3 has
+                // finished, V stage g % 5 once the P V of tile g - 5 has.
+                if (g >= static_cast<uint32_t>(kKStages) &&
+                    !warp_wait(s_full(g % kSBufs), ((g - kKStages) / kSBufs) & 1)) {
                     ok = false;
                     break;
                 }
-                const uint32_t sk = sRing + s * 2 * kKVTileBytes;
+                if (g >= static_cast<uint32_t>(kVStages) &&
+                    !warp_wait(pv_done(g % kVStages), ((g - kVStages) / kVStages) & 1)) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t sk = sK + (g % kKStages) * kKVTileBytes;
+                const uint32_t sv = sV + (g % kVStages) * kKVTileBytes;
+                const uint32_t full = kv_full(g % kKStages);
                 const int r0 = t * kTileN;
                 if (r0 + kTileN <= it.len) {
                     if (lane == 0) {
-                        mbar_arrive_expect_tx(kv_full(s), 2 * kKVTileBytes);
-                        tma_load_3d(sk, &tm_k, 0, it.h, it.start + r0, kv_full(s));
-                        tma_load_3d(sk + kKVTileBytes, &tm_v, 0, it.h, it.start + r0, kv_full(s));
+                        mbar_arrive_expect_tx(full, 2 * kKVTileBytes);
+                        tma_load_3d(sk, &tm_k, 0, it.h, it.start + r0, full);
+                        tma_load_3d(sv, &tm_v, 0, it.h, it.start + r0, full);
                     } else {
-                        mbar_arrive(kv_full(s));
+                        mbar_arrive(full);
                     }
                 } else {
                     warp_load_rows<kTileN>(sk, a.k + seq_off, a.tok_stride, r0, it.len, lane);
-                    warp_load_rows<kTileN>(sk + kKVTileBytes, a.v + seq_off, a.tok_stride, r0, it.len, lane);
-                    publish_copies(kv_full(s));
+                    warp_load_rows<kTileN>(sv, a.v + seq_off, a.tok_stride, r0, it.len, lane);
+                    publish_copies(full);
                 }
             }
         }
         cp_async_wait_all();
         if (*fail_flag) {
             // Let the TMA loads still in flight land before the CTA can exit:
-            // the newest tile of each ring stage and the newest Q loads.
-            for (uint32_t x = g > static_cast<uint32_t>(S) ? g - S : 0; x < g; ++x) mbar_wait(kv_full(x % S), (x / S) & 1);
+            // the newest tile of each K/V barrier and the newest Q loads.
+            for (uint32_t x = g > static_cast<uint32_t>(kKStages) ? g - kKStages : 0; x < g; ++x)
+                mbar_wait(kv_full(x % kKStages), (x / kKStages) & 1);
             for (int x = k > 2 ? k - 2 : 0; x < k; ++x) mbar_wait(q_full(x & 1), (x >> 1) & 1);
         }
     } else if (warp == kMmaWarp) {
@@ -414,63 +449,57 @@ __global__ void __launch_bounds__(kPersistThreads, 2)
         if (lane == 0) {
             const uint32_t idesc_qk = make_idesc(Cvt<T>::kFormat, 0, kTileN);
             const uint32_t idesc_pv = make_idesc(Cvt<T>::kFormat, 1, 64);
-            // P V of tile x (the first of its item when `first`, item index kk).
-            // The stage of an item's last tile is released by the epilogue,
-            // which stages O there.
-            // P V of tile x of item kk: P sits in S buffer x & 1, O in buffer
-            // kk & 1.  An item's first product overwrites its O buffer, which
-            // the epilogue of item kk - 2 must have read out.
-            auto issue_pv = [&](uint32_t x, bool first, bool last, int kk) {
+            // P V of tile x: P sits in S buffer x % 3; the item's first
+            // product overwrites O, which the softmax warps have read out for
+            // the item before (they do so before handing over this tile's P).
+            auto issue_pv = [&](uint32_t x, bool first) {
                 if (!mbar_wait(p_full(x & 3), (x >> 2) & 1)) return false;
-                if (first && kk >= 2 && !mbar_wait(o_empty(kk & 1), ((kk >> 1) - 1) & 1)) return false;
                 fence_after_sync();
-                const uint32_t p_addr = tmem + (x & 1) * static_cast<uint32_t>(kTileN);
-                const uint32_t o_addr = tmem + kOBufCol + (kk & 1) * 64u;
-                const uint32_t sv = sRing + (x % S) * 2 * kKVTileBytes + kKVTileBytes;
+                const uint32_t p_addr = tmem + (x % kSBufs) * static_cast<uint32_t>(kTileN);
+                const uint32_t o_addr = tmem + kOCol;
+                const uint32_t sv = sV + (x % kVStages) * kKVTileBytes;
 #pragma unroll
                 for (int part = 0; part < kParts; ++part)
 #pragma unroll
                     for (int ks = 0; ks < 4; ++ks)
                         mma_f16_ts(o_addr, p_addr + part * 32 + ks * 8, make_sdesc(sv + ks * 2048),
                                    idesc_pv, (first && part == 0 && ks == 0) ? 0u : 1u);
-                mma_commit(pv_done(x & 1));
-                if (!last) mma_commit(kv_empty(x % S));
+                mma_commit(pv_done(x % kVStages));
                 return true;
             };
-            // Two walks over this CTA's tiles: Q K^T runs two tiles ahead of
-            // P V.  P V(g) is issued as soon as P(g) is in TMEM, then Q K^T of
-            // tile g + 2 into S buffer g & 1: the tensor core executes one
+            // Two walks over this CTA's tiles: Q K^T runs three tiles ahead
+            // of P V.  P V(g) is issued as soon as P(g) is in TMEM, then Q K^T
+            // of tile g + 3 into S buffer g % 3: the tensor core executes one
             // thread's MMAs in order, so P V(g) has read P(g) out of that
-            // buffer before the new scores land in it.  The scores of tile
-            // g + 1 are already there, so the softmax never waits for them.
-            Walk wq(blockIdx.x, total, s_cu, s_ip, a.B, a.H);
+            // buffer before the new scores land in it.  The scores of tiles
+            // g + 1 and g + 2 are already there.
+            Walk wq(n_items, s_items, s_cu);
             Walk wp = wq;
             uint32_t gq = 0;
             auto issue_qk = [&]() {
                 const int qb = wq.k & 1;
                 if (wq.t == 0 && !mbar_wait(q_full(qb), (wq.k >> 1) & 1)) return false;
-                const int s = static_cast<int>(gq % S);
-                if (!mbar_wait(kv_full(s), (gq / S) & 1)) return false;
+                if (!mbar_wait(kv_full(gq % kKStages), (gq / kKStages) & 1)) return false;
                 // Tiles filled by cp.async were written through the generic
                 // proxy; order them before the tensor core's reads.
                 fence_async_smem();
                 fence_after_sync();
-                const uint32_t d = tmem + (gq & 1) * static_cast<uint32_t>(kTileN);
+                const uint32_t d = tmem + (gq % kSBufs) * static_cast<uint32_t>(kTileN);
+                const uint32_t sk = sK + (gq % kKStages) * kKVTileBytes;
                 const uint32_t sq = sQ + qb * kQBytes;
-                const uint32_t sk = sRing + s * 2 * kKVTileBytes;
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
                     mma_f16(d, make_sdesc(sq + ks * 32), make_sdesc(sk + ks * 32), idesc_qk, ks > 0);
-                mma_commit(s_full(gq & 1));
+                mma_commit(s_full(gq % kSBufs));
                 if (wq.t == wq.it.nt - 1) mma_commit(q_empty(qb));
                 ++gq;
                 wq.next();
                 return true;
             };
             bool ok = true;
-            for (int i = 0; ok && i < 2 && wq.valid; ++i) ok = issue_qk();
+            for (int i = 0; ok && i < kSBufs && wq.valid; ++i) ok = issue_qk();
             for (uint32_t gp = 0; ok && wp.valid; ++gp) {
-                if (!issue_pv(gp, wp.t == 0, wp.t == wp.it.nt - 1, wp.k)) ok = false;
+                if (!issue_pv(gp, wp.t == 0)) ok = false;
                 else if (wq.valid && !issue_qk()) ok = false;
                 wp.next();
             }
@@ -482,6 +511,7 @@ __global__ void __launch_bounds__(kPersistThreads, 2)
     } else {
         // ---------------- softmax and epilogue (one thread per query row) ----------------
         const uint32_t t_lane = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+        const uint32_t o_lane = t_lane + kOCol;
         // Every product up to tile x has finished.  The phases of each pv_done
         // barrier are waited for one by one, in order: a parity wait is only
         // exact while the barrier is at most one phase behind the target.
@@ -489,101 +519,84 @@ __global__ void __launch_bounds__(kPersistThreads, 2)
         auto confirm_pv = [&](int x) {
             while (pv_seen < x) {
                 ++pv_seen;
-                if (!mbar_wait(pv_done(pv_seen & 1), (pv_seen >> 1) & 1)) {
+                if (!mbar_wait(pv_done(pv_seen % kVStages), (pv_seen / kVStages) & 1)) {
                     atomicExch(&s_fail, 1);
                     pv_seen = x;
                 }
             }
         };
-        // Epilogue of item kk (its last tile gl, running sum lsum): once the
-        // item's last product is done, the K/V stage of tile gl is no longer
-        // read by anything (its release to the load warp is left to this
-        // epilogue), so O / l is staged there: each thread writes its row
-        // (swizzled 16-byte chunks), O buffer kk & 1 is released, and the four
-        // warps store the tile four 128-byte rows per instruction.
-        auto epilogue = [&](const Item& it, int kk, int gl, float lsum) {
+        // This thread's row of O / l, packed to 16-bit pairs, once every
+        // product of the item ending at tile gl has finished.
+        auto read_o = [&](int gl, float lsum, uint32_t (&w)[32]) {
             confirm_pv(gl);
             fence_after_sync();
-            fence_async_smem();
-            const int last_stage = gl % S;
-            uint8_t* stage = smem_raw + (sRing - raw) + last_stage * 2 * kKVTileBytes;
-            if (it.q0 + warp * 32 < it.len) {
-                const float inv = 1.f / lsum;
-                const uint64_t inv2 = f2(inv, inv);
-                const uint32_t o_addr = t_lane + kOBufCol + (kk & 1) * 64u;
+            const float inv = 1.f / lsum;
+            const uint64_t inv2 = f2(inv, inv);
 #pragma unroll
-                for (int hf = 0; hf < 2; ++hf) {
-                    float ov[32];
-                    tmem_ld32(o_addr + hf * 32, ov);
-                    uint32_t w[16];
+            for (int hf = 0; hf < 2; ++hf) {
+                float ov[32];
+                tmem_ld32(o_lane + hf * 32, ov);
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        float o0, o1;
-                        f2_split(f2_mul(f2(ov[2 * i], ov[2 * i + 1]), inv2), o0, o1);
-                        w[i] = Cvt<T>::pack(o0, o1);
-                    }
-#pragma unroll
-                    for (int c = 0; c < 4; ++c)
-                        *reinterpret_cast<uint4*>(stage + swz(tid, hf * 4 + c)) =
-                            make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+                for (int i = 0; i < 16; ++i) {
+                    float o0, o1;
+                    f2_split(f2_mul(f2(ov[2 * i], ov[2 * i + 1]), inv2), o0, o1);
+                    w[hf * 16 + i] = Cvt<T>::pack(o0, o1);
                 }
             }
-            fence_before_sync();
-            mbar_arrive(o_empty(kk & 1));
-            mbar_arrive(o_staged);
-            if (!mbar_wait(o_staged, kk & 1)) {
-                atomicExch(&s_fail, 1);
-                return false;
-            }
-            const int rows = min(kRows, it.len - it.q0);
-            const int c = lane & 7;
-            uint16_t* cls = a.cls_out != nullptr && it.q0 == 0
-                                ? a.cls_out + (static_cast<int64_t>(it.b) * a.H + it.h) * 64
-                                : nullptr;
+        };
+        // Row tid of the item to out (and to cls_out for row 0 of a
+        // sequence), eight 16-byte stores.
+        auto store_o = [&](const Item& it, const uint32_t (&w)[32]) {
+            const int r = it.q0 + tid;
+            if (r >= it.len) return;
+            uint16_t* dst = a.out + static_cast<int64_t>(it.start + r) * a.out_tok_stride + it.h * 64;
+            // 32-byte stores need 32-byte aligned rows (a row stride of a
+            // multiple of 16 elements); 16-byte stores otherwise.  A warp's
+            // store instruction then writes 32 whole sectors instead of 32
+            // half sectors.
+            if ((a.out_tok_stride & 15) == 0 && (reinterpret_cast<uintptr_t>(a.out) & 31) == 0) {
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const int r = i * 16 + warp * 4 + (lane >> 3);
-                if (r < rows) {
-                    const uint4 val = *reinterpret_cast<const uint4*>(stage + swz(r, c));
-                    *reinterpret_cast<uint4*>(a.out + static_cast<int64_t>(it.start + it.q0 + r) * a.out_tok_stride +
-                                              it.h * 64 + c * 8) = val;
-                    if (r == 0 && cls != nullptr) *reinterpret_cast<uint4*>(cls + c * 8) = val;
-                }
+                for (int c = 0; c < 4; ++c)
+                    asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(dst + c * 16),
+                                 "r"(w[8 * c]), "r"(w[8 * c + 1]), "r"(w[8 * c + 2]), "r"(w[8 * c + 3]),
+                                 "r"(w[8 * c + 4]), "r"(w[8 * c + 5]), "r"(w[8 * c + 6]), "r"(w[8 * c + 7])
+                                 : "memory");
+            } else {
+#pragma unroll
+                for (int c = 0; c < 8; ++c)
+                    *reinterpret_cast<uint4*>(dst + c * 8) =
+                        make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
             }
-            // The stage goes back to the load warp once every read of it is done.
-            fence_async_smem();
-            mbar_arrive(o_stored);
-            if (tid == 0) {
-                if (mbar_wait(o_stored, kk & 1)) mbar_arrive(kv_empty(last_stage));
-                else atomicExch(&s_fail, 1);
+            if (a.cls_out != nullptr && r == 0) {
+                uint16_t* cls = a.cls_out + (static_cast<int64_t>(it.b) * a.H + it.h) * 64;
+#pragma unroll
+                for (int c = 0; c < 8; ++c)
+                    *reinterpret_cast<uint4*>(cls + c * 8) =
+                        make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
             }
-            return true;
         };
         const uint64_t sl2 = f2(a.scale_log2, a.scale_log2);
-        // The epilogue of an item runs after the first tile of the next one,
-        // by when its last product has long finished.
+        // The epilogue of an item runs at the first tile of the next one,
+        // before that tile's P is handed over (the next product overwrites O).
         bool pending = false;
         Item p_it{};
-        int p_k = 0, p_gl = 0;
+        int p_gl = 0;
         float p_l = 0.f;
         int g = 0;
-        int k = 0;
         bool ok = true;
-        for (int j = blockIdx.x; ok && j < total; j += gridDim.x, ++k) {
-            if (*fail_flag) break;
-            const Item it = decode_item(j, s_cu, s_ip, a.B, a.H);
+        for (int k = 0; ok && k < n_items; ++k) {
+            const Item it = unpack_item(s_items[k], s_cu);
             const bool warp_rows = it.q0 + warp * 32 < it.len;
-            const uint32_t o_buf = t_lane + kOBufCol + (k & 1) * 64u;
             float m_ref = -INFINITY;   // reference maximum (log2 units) of this row
             float l0 = 0.f, l1 = 0.f;  // running sum, even / odd keys
             for (int t = 0; t < it.nt; ++t, ++g) {
-                if (!mbar_wait(s_full(g & 1), (g >> 1) & 1)) {
+                if (!mbar_wait(s_full(g % kSBufs), (g / kSBufs) & 1)) {
                     atomicExch(&s_fail, 1);
                     ok = false;
                     break;
                 }
                 fence_after_sync();
-                const uint32_t s_buf = t_lane + static_cast<uint32_t>((g & 1) * kTileN);
+                const uint32_t s_buf = t_lane + static_cast<uint32_t>((g % kSBufs) * kTileN);
                 if (warp_rows) {
                     float sv[64];
                     tmem_ld64(s_buf, sv);
@@ -621,11 +634,11 @@ __global__ void __launch_bounds__(kPersistThreads, 2)
 #pragma unroll
                         for (int q = 0; q < 4; ++q) {
                             float part[16];
-                            tmem_ld16(o_buf + q * 16, part);
+                            tmem_ld16(o_lane + q * 16, part);
 #pragma unroll
                             for (int i = 0; i < 8; ++i)
                                 f2_split(f2_mul(f2(part[2 * i], part[2 * i + 1]), a2), part[2 * i], part[2 * i + 1]);
-                            tmem_st16(o_buf + q * 16, part);
+                            tmem_st16(o_lane + q * 16, part);
                         }
                     }
                     // P(g) replaces S(g) in its TMEM buffer: the product that
@@ -660,29 +673,37 @@ __global__ void __launch_bounds__(kPersistThreads, 2)
                     f2_split(lsum, l0, l1);
                     tmem_wait_st();
                 }
-                // Every warp, rows or not, takes each pv_done phase while it is
-                // the barrier's next one (products up to g - 2 are long done).
-                // This comes before the arrival for tile g: after it, P V(g)
-                // may complete and move barrier g & 1 one phase past g - 2.
-                if (g >= 2) confirm_pv(g - 2);
-                fence_before_sync();
-                mbar_arrive(p_full(g & 3));
                 if (t == 0 && pending) {
-                    if (!epilogue(p_it, p_k, p_gl, p_l)) {
-                        ok = false;
-                        break;
+                    // The previous item's O, read out and stored before this
+                    // tile's P is handed over: its first product overwrites O.
+                    if (p_it.q0 + warp * 32 < p_it.len) {
+                        uint32_t ow[32];
+                        read_o(p_gl, p_l, ow);
+                        store_o(p_it, ow);
+                    } else {
+                        confirm_pv(p_gl);
                     }
                     pending = false;
                 }
+                // Every warp, rows or not, takes each pv_done phase while it is
+                // the barrier's next one (products up to g - 2 are long done).
+                // This comes before the arrival for tile g: after it, P V(g)
+                // may complete and move barrier g % 5 one phase past g - 5.
+                if (g >= 2) confirm_pv(g - 2);
+                fence_before_sync();
+                mbar_arrive(p_full(g & 3));
             }
             if (!ok || *fail_flag) break;
             pending = true;
             p_it = it;
-            p_k = k;
             p_gl = g - 1;
             p_l = l0 + l1;
         }
-        if (ok && pending && !*fail_flag) epilogue(p_it, p_k, p_gl, p_l);
+        if (ok && pending && !*fail_flag && p_it.q0 + warp * 32 < p_it.len) {
+            uint32_t ow[32];
+            read_o(p_gl, p_l, ow);
+            store_o(p_it, ow);
+        }
     }
 
     fence_before_sync();

@@ -251,7 +251,13 @@ ragged_status launch_tc05_persist(const ragged::resident::PackedRows& src, int64
     using namespace ragged::tc05;
     *launched = false;
     const int64_t q_tiles = (max_seqlen + kRows - 1) / kRows;
-    if (B > kPersistMaxB || B * H * q_tiles >= (int64_t(1) << 31)) return RAGGED_OK;
+    // Items are packed into 32-bit words (sequence: 11 bits, head: 10, query
+    // tile: 11), and each CTA keeps at most kPersistMaxItems of them.
+    if (B > kPersistMaxB || H > 1023 || q_tiles > 2047) return RAGGED_OK;
+    const int64_t items_bound = B * H * q_tiles;
+    const int64_t ctas = std::min<int64_t>(items_bound, 2LL * sm_count());
+    const int64_t items_cap = (items_bound + ctas - 1) / ctas;
+    if (items_cap > kPersistMaxItems) return RAGGED_OK;
     // Full tiles never reach past the last row of their sequence, and every
     // sequence ends within B * max_seqlen rows.
     const int64_t rows = B * max_seqlen;
@@ -261,15 +267,14 @@ ragged_status launch_tc05_persist(const ragged::resident::PackedRows& src, int64
         !tensor_map_3d(&tv, src.v, H, rows, src.head_stride, src.tok_stride, kTileN))
         return RAGGED_OK;
     auto kernel = attn_tc05_persist_kernel<T>;
-    ragged_status st = ensure_smem(kernel, persist_smem_bytes(kPersistMaxB), g_persist_smem[slot]);
+    ragged_status st = ensure_smem(kernel, persist_smem_bytes(kPersistMaxB, kPersistMaxItems), g_persist_smem[slot]);
     if (st != RAGGED_OK) return st;
-    const int64_t items_bound = B * H * q_tiles;
-    const int64_t ctas = std::min<int64_t>(items_bound, 2LL * sm_count());
     PersistArgs args{src.q, src.k, src.v, src.tok_stride, src.head_stride, src.cu, static_cast<int>(B),
                      static_cast<int>(H), static_cast<int>(max_seqlen), scale * 1.4426950408889634f,
-                     static_cast<uint16_t*>(out), out_tok_stride, static_cast<uint16_t*>(cls_out)};
-    kernel<<<static_cast<unsigned>(ctas), kPersistThreads, persist_smem_bytes(static_cast<int>(B)), s>>>(tq, tk, tv,
-                                                                                                        args);
+                     static_cast<uint16_t*>(out), out_tok_stride, static_cast<uint16_t*>(cls_out),
+                     static_cast<int>(items_cap)};
+    kernel<<<static_cast<unsigned>(ctas), kPersistThreads,
+             persist_smem_bytes(static_cast<int>(B), static_cast<int>(items_cap)), s>>>(tq, tk, tv, args);
     *launched = true;
     return cuda_check(cudaGetLastError(), "persistent tcgen05 attention launch");
 }
