@@ -191,10 +191,12 @@ RAGGED_API int32_t ragged_set_attn_kernel(int32_t kernel);
  * The decision is exact, whatever the order of summation: a token is kept
  * when sum(x_c^2) >= tau^2 in exact arithmetic, CLS always.  With tau <= 0
  * every token is kept except those with a NaN element, which are always
- * dropped; a token with an infinite element (and no NaN) is always kept.  An
- * fp64 sum settles the bit unless it lies within a relative 2^-26 of tau^2;
- * there one lane forms the sum exactly, as an integer multiple of 2^-298,
- * which costs O(C) serial steps for that token.
+ * dropped; a token with an infinite element (and no NaN) is always kept.  A
+ * sum within a relative 2^-29 of the exact one (fp32 squares with error-free
+ * two-sum accumulation for f16 / bf16 rows on 16-byte boundaries with C a
+ * multiple of 8 up to 8192, else fp64) settles the bit unless it lies within
+ * a relative 2^-26 of tau^2; there one lane forms the sum exactly, as an
+ * integer multiple of 2^-298, which costs O(C) serial steps for that token.
  */
 RAGGED_API ragged_status ragged_mask_l2(const void *x, int64_t B, int64_t L_full, int64_t C, int64_t tok_stride,
                                         ragged_dtype dtype, double tau, uint8_t *keep, void *stream);

@@ -15,6 +15,8 @@
 // itself, so selection, cu_seqlens and the survivor copy are one launch.
 #pragma once
 
+#include <type_traits>
+
 #include "pack.cuh"
 
 namespace ragged {
@@ -157,6 +159,105 @@ __global__ void __launch_bounds__(kMaskThreads)
         else kept = lane == 0 ? l2_exact_reaches<T>(x, base, C, tau) : false;
     }
     if (lane == 0) keep[t] = kept ? 1 : 0;
+}
+
+// ---- vector path for f16 / bf16 rows -----------------------------------------
+//
+// Used when the rows are 16-byte aligned (x and tok_stride * 2), C is a
+// multiple of 8 and at most kMaskVecMaxC.  One half-warp per token, each lane
+// reading whole 16-byte vectors (8 elements).  A square of an f16 or bf16
+// value is exact in fp32 unless it leaves fp32's normal range (only bf16 can),
+// and each lane adds its squares into two fp32 accumulators with an
+// error-free two-sum, keeping the rounding errors in a second pair: with n
+// terms per accumulator the pair (s, c) is within a relative n^2 2^-48 of its
+// exact sum (n = C / 32 <= 256 here: 2^-32).  The 32 pairs of a token are then added in
+// fp64 (a relative 2^-48 more).  That sum is trusted where it is finite and
+// at least 2^-100 (squares below fp32's normal range then add at most a
+// relative 2^-37; f16 squares never leave it, so an f16 sum of 0 is exact
+// too); elsewhere (NaN, an infinite element, a bf16 overflow or underflow)
+// the token falls back to the fp64 sum of mask_l2_kernel.  The decision is
+// the same as there, on a sum within a relative 2^-29 of the exact one.
+constexpr int kMaskVecMaxC = 8192;   // at most 256 terms per accumulator
+
+__device__ __forceinline__ void two_sum_acc(float& s, float& c, float y) {
+    const float t = __fadd_rn(s, y);
+    const float bp = __fsub_rn(t, s);
+    const float e = __fadd_rn(__fsub_rn(s, __fsub_rn(t, bp)), __fsub_rn(y, bp));
+    s = t;
+    c = __fadd_rn(c, e);
+}
+
+template <typename T>
+__device__ __forceinline__ float2 widen2(uint32_t w);
+template <>
+__device__ __forceinline__ float2 widen2<__half>(uint32_t w) {
+    return __half22float2(*reinterpret_cast<const __half2*>(&w));
+}
+template <>
+__device__ __forceinline__ float2 widen2<__nv_bfloat16>(uint32_t w) {
+    return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kMaskThreads)
+    mask_l2_vec_kernel(const void* __restrict__ x, int L_full, int C, int64_t tok_stride, double tau,
+                       uint8_t* __restrict__ keep) {
+    const int j = blockIdx.x * (kMaskThreads / 16) + (threadIdx.x >> 4);
+    const int hl = threadIdx.x & 15;                    // lane within the half-warp
+    const unsigned hmask = 0xffffu << (threadIdx.x & 16);
+    if (j >= L_full) return;   // uniform over the half-warp
+    const int64_t t = static_cast<int64_t>(blockIdx.y) * L_full + j;
+    const int64_t base = t * tok_stride;
+    const uint4* row = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(x) + base);
+    const int nvec = C >> 3;
+    float s0 = 0.f, c0 = 0.f, s1 = 0.f, c1 = 0.f;
+    // Four vectors per lane in flight before any arithmetic (vectors past the
+    // row read as zeros, whose squares add nothing).  Two or four tokens per
+    // half-warp, with all their vectors in flight, measured slower.
+    constexpr int kVecs = 4;
+    for (int v0 = hl; v0 < nvec; v0 += 16 * kVecs) {
+        uint4 q[kVecs];
+#pragma unroll
+        for (int k = 0; k < kVecs; ++k) q[k] = v0 + 16 * k < nvec ? __ldg(row + v0 + 16 * k) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+        for (int k = 0; k < kVecs; ++k) {
+            const uint32_t w[4] = {q[k].x, q[k].y, q[k].z, q[k].w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float2 f = widen2<T>(w[i]);
+                two_sum_acc(s0, c0, __fmul_rn(f.x, f.x));
+                two_sum_acc(s1, c1, __fmul_rn(f.y, f.y));
+            }
+        }
+    }
+    double ss = __dadd_rn(__dadd_rn(static_cast<double>(s0), static_cast<double>(c0)),
+                          __dadd_rn(static_cast<double>(s1), static_cast<double>(c1)));
+#pragma unroll
+    for (int off = 8; off > 0; off >>= 1) ss = __dadd_rn(ss, __shfl_xor_sync(hmask, ss, off));
+    const bool trusted = isfinite(ss) && (ss >= 0x1p-100 || (ss == 0.0 && std::is_same<T, __half>::value));
+    if (!trusted) {   // uniform over the half-warp: the fp64 sum of mask_l2_kernel
+        double acc = 0.0;
+        for (int c = hl; c < C; c += 16) {
+            const double v = widen<T>(x, base + c);
+            acc = __dadd_rn(acc, __dmul_rn(v, v));
+        }
+#pragma unroll
+        for (int off = 8; off > 0; off >>= 1) acc = __dadd_rn(acc, __shfl_xor_sync(hmask, acc, off));
+        ss = acc;
+    }
+    bool kept;
+    if (j == 0) kept = true;
+    else if (isnan(ss)) kept = false;
+    else if (isinf(ss) || !(tau > 0.0)) kept = true;
+    else if (tau > 0x1p+140) kept = false;
+    else if (tau < 0x1p-400) kept = ss > 0.0;
+    else {
+        const double t2 = __dmul_rn(tau, tau);
+        if (ss > __dmul_rn(t2, 1.0 + 0x1p-26)) kept = true;
+        else if (ss < __dmul_rn(t2, 1.0 - 0x1p-26)) kept = false;
+        else kept = hl == 0 ? l2_exact_reaches<T>(x, base, C, tau) : false;
+    }
+    if (hl == 0) keep[t] = kept ? 1 : 0;
 }
 
 // The top-k order as one unsigned key per token, larger key = ranks earlier:

@@ -400,13 +400,22 @@ ragged_status ragged_mask_l2(const void* x, int64_t B, int64_t L_full, int64_t C
     if (reinterpret_cast<uintptr_t>(x) % esz) return fail(RAGGED_ERR_INVALID_ARG, "x is not element-aligned");
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int L = static_cast<int>(L_full), Ci = static_cast<int>(C);
-    const unsigned chunks = static_cast<unsigned>((L_full + ragged::kMaskThreads / 32 - 1) / (ragged::kMaskThreads / 32));
+    // 16-bit rows that start on 16-byte boundaries go through the vector path
+    // (one half-warp per token, 16-byte loads, fp32 two-sum accumulation).
+    const bool vec = esz == 2 && aligned16(x) && (tok_stride * 2) % 16 == 0 && C % 8 == 0 && C <= ragged::kMaskVecMaxC;
+    const int per_cta = vec ? ragged::kMaskThreads / 16 : ragged::kMaskThreads / 32;
+    const unsigned chunks = static_cast<unsigned>((L_full + per_cta - 1) / per_cta);
     for (int64_t b0 = 0; b0 < B; b0 += ragged::kMaskMaxImages) {
         const int64_t nb = B - b0 < ragged::kMaskMaxImages ? B - b0 : ragged::kMaskMaxImages;
         const dim3 grid(chunks, static_cast<unsigned>(nb));
         const void* xb = static_cast<const char*>(x) + b0 * L_full * tok_stride * esz;
         uint8_t* kb = keep + b0 * L_full;
-        if (dtype == RAGGED_F16)
+        if (vec && dtype == RAGGED_F16)
+            ragged::mask_l2_vec_kernel<__half><<<grid, ragged::kMaskThreads, 0, s>>>(xb, L, Ci, tok_stride, tau, kb);
+        else if (vec)
+            ragged::mask_l2_vec_kernel<__nv_bfloat16><<<grid, ragged::kMaskThreads, 0, s>>>(xb, L, Ci, tok_stride, tau,
+                                                                                           kb);
+        else if (dtype == RAGGED_F16)
             ragged::mask_l2_kernel<__half><<<grid, ragged::kMaskThreads, 0, s>>>(xb, L, Ci, tok_stride, tau, kb);
         else if (dtype == RAGGED_BF16)
             ragged::mask_l2_kernel<__nv_bfloat16><<<grid, ragged::kMaskThreads, 0, s>>>(xb, L, Ci, tok_stride, tau, kb);

@@ -91,6 +91,52 @@ def test_mask_l2_on_a_strided_view():
     assert np.array_equal(got, oracle.mask_l2(np.ascontiguousarray(qn), w.dtype, tau))
 
 
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+def test_mask_l2_vector_path_special_values(dtype):
+    """16-bit rows on 16-byte boundaries take the vector path (fp32 squares,
+    two-sum accumulation): tokens whose sum it cannot trust (NaN, an infinite
+    element, bf16 squares above or below fp32's range, all zeros) go back to the
+    fp64 sum, and a near-tie still reaches the exact comparison."""
+    big, tiny = (2.0 ** 70, 2.0 ** -80) if dtype == "bf16" else (65504.0, 2.0 ** -24)
+    x = np.zeros((1, 10, 64), dtype=np.float32)
+    x[0, 1, :3] = big                          # bf16: squares overflow fp32
+    x[0, 2, :40] = tiny                        # bf16: squares underflow fp32
+    x[0, 3, 0] = 1.0
+    x[0, 3, 1:33] = 2.0 ** -70 if dtype == "bf16" else 2.0 ** -24    # 1 plus tiny squares
+    x[0, 4, 5], x[0, 4, 6] = np.nan, 3.0
+    x[0, 5, 9] = np.inf
+    x[0, 7, :] = 0.625                         # norm 5 exactly
+    x[0, 8, :] = -0.625
+    x[0, 9, ::2] = 1.5
+    xs = synthetic.store(x, dtype)
+    xd = to_device(xs, dtype)
+    xf = oracle.decode(xs, dtype).reshape(1, 10, 64)
+    norms = np.sqrt((xf.astype(np.float64) ** 2).sum(2))
+    taus = [0.0, -1.0, 5.0, float(np.nextafter(5.0, 0.0)), float(np.nextafter(5.0, 6.0)), 1.0,
+            float(np.nextafter(1.0, 2.0)), float(big), float(tiny), 1e-300, 1e300, float("inf")]
+    taus += [float(v) for v in norms[0] if np.isfinite(v) and v > 0]
+    for tau in taus:
+        got = rv.ragged_mask_l2(xd, tau).cpu().numpy()
+        assert np.array_equal(got, oracle.mask_l2(xs, dtype, tau)), tau
+
+
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+def test_mask_l2_rows_off_16_byte_boundaries(dtype):
+    """A view starting one element into its buffer (rows on 2-byte boundaries)
+    takes the per-element path; both paths give the oracle's mask."""
+    rng = synthetic.rng_for(3011, ["f16", "bf16"].index(dtype))
+    B, L, C = 3, 50, 128
+    x = synthetic.store(rng.standard_normal((B, L, C + 8)).astype(np.float32), dtype)
+    full = to_device(x, dtype)                                 # [B, L, C + 8]
+    for off in (0, 1):
+        view = full[:, :, off:off + C]
+        xs = np.ascontiguousarray(x[:, :, off:off + C])
+        xf = oracle.decode(xs, dtype).reshape(B, L, C)
+        tau = float(np.median(np.sqrt((xf.astype(np.float64) ** 2).sum(2))))
+        got = rv.ragged_mask_l2(view, tau).cpu().numpy()
+        assert np.array_equal(got, oracle.mask_l2(xs, dtype, tau)), off
+
+
 def _topk_case(rng, B, L, ties, nans):
     s = rng.standard_normal((B, L)).astype(np.float32)
     if ties:
