@@ -211,23 +211,16 @@ __global__ void __launch_bounds__(kMaskThreads)
     const uint4* row = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(x) + base);
     const int nvec = C >> 3;
     float s0 = 0.f, c0 = 0.f, s1 = 0.f, c1 = 0.f;
-    // Four vectors per lane in flight before any arithmetic (vectors past the
-    // row read as zeros, whose squares add nothing).  Two or four tokens per
-    // half-warp, with all their vectors in flight, measured slower.
-    constexpr int kVecs = 4;
-    for (int v0 = hl; v0 < nvec; v0 += 16 * kVecs) {
-        uint4 q[kVecs];
+    // One vector per lane and step.  Requesting four vectors before any
+    // arithmetic, or two or four tokens per half-warp, measured slower.
+    for (int v = hl; v < nvec; v += 16) {
+        const uint4 q = __ldg(row + v);
+        const uint32_t w[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
-        for (int k = 0; k < kVecs; ++k) q[k] = v0 + 16 * k < nvec ? __ldg(row + v0 + 16 * k) : make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll
-        for (int k = 0; k < kVecs; ++k) {
-            const uint32_t w[4] = {q[k].x, q[k].y, q[k].z, q[k].w};
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const float2 f = widen2<T>(w[i]);
-                two_sum_acc(s0, c0, __fmul_rn(f.x, f.x));
-                two_sum_acc(s1, c1, __fmul_rn(f.y, f.y));
-            }
+        for (int i = 0; i < 4; ++i) {
+            const float2 f = widen2<T>(w[i]);
+            two_sum_acc(s0, c0, __fmul_rn(f.x, f.x));
+            two_sum_acc(s1, c1, __fmul_rn(f.y, f.y));
         }
     }
     double ss = __dadd_rn(__dadd_rn(static_cast<double>(s0), static_cast<double>(c0)),
