@@ -351,6 +351,17 @@ def test_persistent_above_its_batch_limit(dtype):
     check_against_oracle(w, seqs=sample_sequences(w.lengths, 12, seed=3), kernel="persistent")
 
 
+@pytest.mark.parametrize("H", [1023, 1024])
+def test_persistent_at_its_head_limit(H):
+    """A packed work item holds a head index of 10 bits: H = 1023 runs the
+    persistent kernel with every head index in use, H = 1024 runs the per-tile
+    tcgen05 kernel instead; both match the oracle on every sequence."""
+    rng = np.random.default_rng(88)
+    lengths = np.array([70, 1, 129])
+    w = synthetic.make_workload("heads", 3, 130, H, lengths, "f16", 88)
+    check_against_oracle(w, kernel="persistent")
+
+
 @pytest.mark.parametrize("dtype", ["f16", "bf16"])
 def test_persistent_many_items_per_cta(dtype):
     """Several items per CTA with every length class (full and partial query
