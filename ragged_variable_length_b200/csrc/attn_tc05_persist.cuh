@@ -329,13 +329,23 @@ __global__ void __launch_bounds__(kPersistThreads, 2)
     fence_before_sync();
     __syncthreads();
     fence_after_sync();
-    if (warp == kLoadWarp) {   // item offsets: warp-wide inclusive scans over 32 sequences at a time
-        int carry = 0;
-        if (lane == 0) s_ip[0] = 0;
-        for (int c0 = 0; c0 < a.B; c0 += 32) {
-            const int b = c0 + lane;
-            int n = 0;
-            if (b < a.B) {
+    // Item offsets: s_ip[b] = items of the sequences before b.  Every thread
+    // takes a contiguous run of at most six sequences (B <= 1024), and the run
+    // totals are scanned across the block (a warp scan, then the six warp
+    // totals), so the scan takes a few shared-memory round trips whatever B
+    // is; one warp walking 32 sequences at a time took ~3 us at B = 512.
+    {
+        constexpr int kWarps = kPersistThreads / 32;
+        __shared__ int s_wsum[kWarps];
+        const int per = (a.B + kPersistThreads - 1) / kPersistThreads;
+        const int b0 = min(a.B, tid * per), b1 = min(a.B, b0 + per);
+        int n[(kPersistMaxB + kPersistThreads - 1) / kPersistThreads];
+        int run = 0;
+#pragma unroll
+        for (int i = 0; i < (kPersistMaxB + kPersistThreads - 1) / kPersistThreads; ++i) {
+            const int b = b0 + i;
+            n[i] = 0;
+            if (b < b1) {
                 const int st = s_cu[b], len = s_cu[b + 1] - st;
                 // The tensor maps cover rows [0, B * max_seqlen): a sequence
                 // reaching past them (cu[0] != 0 can shift one there) would
@@ -343,15 +353,29 @@ __global__ void __launch_bounds__(kPersistThreads, 2)
                 if (st < 0 || len < 0 || len > a.max_seqlen ||
                     static_cast<int64_t>(st) + len > static_cast<int64_t>(a.B) * a.max_seqlen)
                     raise_status(RAGGED_DEV_BAD_SEQLENS);
-                else n = ((len + kRows - 1) / kRows) * a.H;
+                else
+                    n[i] = ((len + kRows - 1) / kRows) * a.H;
+                run += n[i];
             }
+        }
+        int incl = run;   // inclusive scan of the run totals within the warp
 #pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int y = __shfl_up_sync(kFullMask, n, o);
-                if (lane >= o) n += y;
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(kFullMask, incl, o);
+            if (lane >= o) incl += y;
+        }
+        if (lane == 31) s_wsum[warp] = incl;
+        __syncthreads();
+        int before = incl - run;
+        for (int w = 0; w < warp; ++w) before += s_wsum[w];
+        if (tid == 0) s_ip[0] = 0;
+#pragma unroll
+        for (int i = 0; i < (kPersistMaxB + kPersistThreads - 1) / kPersistThreads; ++i) {
+            const int b = b0 + i;
+            if (b < b1) {
+                before += n[i];
+                s_ip[b + 1] = before;
             }
-            if (b < a.B) s_ip[b + 1] = carry + n;
-            carry += __shfl_sync(kFullMask, n, 31);
         }
     }
     __syncthreads();
